@@ -156,8 +156,11 @@ vq_status vq_moe_grouped(const vq_matrix *gate, const vq_matrix *up, const vq_ma
                          const float *expert_w, int32_t topk, void *y, vq_dtype yt,
                          void *ws, size_t ws_bytes, vq_stream_t stream);
 
-/* Synchronise `stream` and read the status word a vq_moe_grouped call left in ws:
- * VQ_OK, VQ_ERR_DEVICE_FLAG (bad expert ids seen) or VQ_ERR_CUDA. */
+/* Synchronise `stream`, then report what the device recorded: VQ_ERR_TIMEOUT if any
+ * kernel of this library gave up a bounded wait since the library was loaded (a bug
+ * signal; the kernel ended instead of hanging), else, when ws is not NULL, the status
+ * word a vq_moe_grouped call left in ws: VQ_ERR_DEVICE_FLAG if it skipped expert ids
+ * outside [0, E); VQ_OK otherwise.  VQ_ERR_CUDA if the synchronisation failed. */
 vq_status vq_read_device_status(const void *ws, vq_stream_t stream);
 
 /* Static description of a status code (never NULL). */

@@ -128,13 +128,15 @@ def unpack(packed: np.ndarray, ncodes: int, bits: int, L=None) -> np.ndarray:
 class Tensor:
     """A VQ tensor in the oracle's own packed form (packed by `pack` above)."""
 
-    def __init__(self, data, L=None):
+    def __init__(self, data, L=None, experts=None):
+        """`experts`: pack only these experts (the others stay zero) — for full-size
+        checks that evaluate a sample of tokens."""
         self.L = L or lib()
         self.data = data
         E, rows = data.num_experts, data.rows
         self.row_bytes = code_row_bytes(data.ncodes, data.bits, self.L)
-        self.codes = np.empty((E, rows, self.row_bytes), np.uint8)
-        for e in range(E):
+        self.codes = np.zeros((E, rows, self.row_bytes), np.uint8)
+        for e in (range(E) if experts is None else sorted(set(int(v) for v in experts))):
             self.codes[e] = pack(data.codes[e], data.bits, self.row_bytes, self.L)
         self.codebook = np.ascontiguousarray(data.codebook, dtype=np.uint16)
         self.scales = np.ascontiguousarray(data.scales, dtype=np.uint16)

@@ -1,0 +1,415 @@
+// vq_gemm.cu — prefill GEMM y[m][n] = sum_k x[m][k] W[n][k] on the tcgen05 tensor cores,
+// with W expanded from its VQ codes inside the kernel.
+//
+// The pages' prefill path (paper "Data-Free Vector Quantization Beats Affine Quantization
+// at Matched Bytes Below 5 Bits", §2.5 and §3.4: the prefill-shaped code path and the
+// fused decode-and-matmul) is a dense contraction once the weights are expanded, so on
+// sm_100a it runs on the 5th-generation tensor cores:
+//
+//   * one CTA computes a 128 (weight rows) x BT (tokens) output tile; the weight tile is
+//     the MMA's A operand (M = 128), the activation tile its B operand (N = BT), so each
+//     expanded weight is used by BT tokens;
+//   * warp 0 (one thread) streams activation tiles [BT][64] into shared memory with TMA
+//     (128-byte swizzle);
+//   * warps 2-5 (128 threads, one weight row each) read the row's packed codes and its
+//     scale for the next 64 columns straight from global memory, look the codes up in
+//     the shared-memory codebook, multiply by the scale (one rounding to the tile type)
+//     and write the 128 x 64 tile in the same 128-byte-swizzled K-major layout, then
+//     fence the generic->async proxy and signal an mbarrier;
+//   * warp 1 (one thread) issues tcgen05.mma (kind::f16, fp32 accumulation in tensor
+//     memory) for each 64-column stage and frees the stage with tcgen05.commit;
+//   * after the last stage, warps 2-5 read the accumulator out of tensor memory
+//     (tcgen05.ld) and store y.
+// Stages are a ring of STAGES buffers guarded by mbarriers; every wait is bounded and a
+// wait that runs out sets the library's device error word instead of hanging.
+#include <algorithm>
+
+#include "vq_codebook.cuh"
+#include "vq_internal.cuh"
+#include "vq_sm100.cuh"
+
+namespace vq {
+
+__device__ unsigned int g_device_error;   // nonzero after a bounded wait ran out
+
+constexpr int GEMM_BM = 128;       // weight rows per tile (UMMA M)
+constexpr int GEMM_BK = 64;        // columns per stage (one 128-byte swizzle row of 16-bit)
+constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 expansion + epilogue
+constexpr int A_TILE_BYTES = GEMM_BM * GEMM_BK * 2;
+
+// Packed codes of one row for one 64-column stage: 64/d codes.
+template <int D, int BITS>
+struct CodeBlock {
+    static constexpr int BYTES = (64 / D) * BITS / 8;   // 32, 16, 8 (8-bit); 48, 24, 12 (12-bit)
+    static constexpr int WORDS = BYTES / 4;
+    uint32_t w[WORDS];
+
+    __device__ __forceinline__ void load(const uint8_t *row, int kb) {
+        const uint8_t *p = row + (int64_t)kb * BYTES;
+        if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+            for (int v = 0; v < BYTES / 16; v++) {
+                uint4 u = ldg_stream_u4(p + 16 * v);
+                w[4 * v] = u.x; w[4 * v + 1] = u.y; w[4 * v + 2] = u.z; w[4 * v + 3] = u.w;
+            }
+        } else if constexpr (BYTES % 8 == 0) {
+#pragma unroll
+            for (int v = 0; v < BYTES / 8; v++) {
+                uint2 u = __ldg(reinterpret_cast<const uint2 *>(p) + v);
+                w[2 * v] = u.x; w[2 * v + 1] = u.y;
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < WORDS; v++) w[v] = __ldg(reinterpret_cast<const uint32_t *>(p) + v);
+        }
+    }
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int v = 0; v < WORDS; v++) w[v] = 0u;
+    }
+    __device__ __forceinline__ uint32_t code(int q) const {
+        if constexpr (BITS == 8) {
+            return (w[q >> 2] >> ((q & 3) * 8)) & 0xFFu;
+        } else {
+            const int bit = 12 * q, wi = bit >> 5, sh = bit & 31;
+            if (sh + 12 <= 32) return (w[wi] >> sh) & 0xFFFu;
+            return __funnelshift_r(w[wi], w[wi + 1], sh) & 0xFFFu;
+        }
+    }
+};
+
+// scale * (two fp16 codebook values) -> two tile elements, one rounding.
+template <bool BF16T>
+__device__ __forceinline__ uint32_t scale_pair(uint32_t cb2, __half2 s2, float sf) {
+    if constexpr (!BF16T) {
+        __half2 r = __hmul2(*reinterpret_cast<__half2 *>(&cb2), s2);
+        return *reinterpret_cast<uint32_t *>(&r);
+    } else {
+        float2 f = __half22float2(*reinterpret_cast<__half2 *>(&cb2));
+        __nv_bfloat162 r = __floats2bfloat162_rn(f.x * sf, f.y * sf);
+        return *reinterpret_cast<uint32_t *>(&r);
+    }
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ void flag_error(volatile int *abort_flag) {
+    *abort_flag = 1;
+    atomicExch(&g_device_error, 1u);
+}
+
+template <int D, int BITS, int BT, int STAGES, bool BF16T>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, Mat W, int M, void *__restrict__ y, int yt)
+{
+    using CB = SmemCB<D, BITS>;
+    using Blk = CodeBlock<D, BITS>;
+    constexpr int B_TILE_BYTES = BT * GEMM_BK * 2;
+    constexpr uint32_t TMEM_COLS = BT;          // fp32 accumulator: one column per token
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + STAGES * A_TILE_BYTES;
+    uint8_t *sCB = sB + STAGES * B_TILE_BYTES;
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(sCB + CB::BYTES);
+    uint64_t *full_b = full_a + STAGES;
+    uint64_t *empty = full_b + STAGES;
+    uint64_t *acc_bar = empty + STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *consumed = reinterpret_cast<volatile int *>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BT;
+    const int n0 = blockIdx.y * GEMM_BM;
+    const int nkb = W.cols / GEMM_BK;
+
+    CB::stage(sCB, W.codebook);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; s++) {
+            mbar_init(&full_a[s], 4);
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_bar, 1);
+        *abort_flag = 0;
+        *consumed = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer: activation tiles
+        if (lane == 0) {
+            tma_prefetch_map(&xmap);
+            int issued = 0;
+            for (int kb = 0; kb < nkb; kb++) {
+                const int s = kb % STAGES, r = kb / STAGES;
+                if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1)) { flag_error(abort_flag); break; }
+                if (*abort_flag) break;
+                mbar_arrive_expect_tx(&full_b[s], B_TILE_BYTES);
+                tma_load_2d(sB + s * B_TILE_BYTES, &xmap, &full_b[s], kb * GEMM_BK, m0);
+                issued++;
+            }
+            // On an abort, wait (bounded) for the loads still in flight before leaving.
+            if (*abort_flag) {
+                for (int kb = *consumed; kb < issued; kb++)
+                    mbar_wait(&full_b[kb % STAGES], (kb / STAGES) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16(GEMM_BM, BT, BF16T);
+            for (int kb = 0; kb < nkb; kb++) {
+                const int s = kb % STAGES, r = kb / STAGES;
+                if (!mbar_wait(&full_a[s], r & 1) || !mbar_wait(&full_b[s], r & 1)) {
+                    flag_error(abort_flag);
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t adesc = smem_desc_sw128(smem_u32(sA + s * A_TILE_BYTES));
+                const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * B_TILE_BYTES));
+#pragma unroll
+                for (int k = 0; k < GEMM_BK / 16; k++)   // K = 16 per MMA: +32 bytes = +2 in the address field
+                    umma_f16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&empty[s]);
+                *consumed = kb + 1;
+            }
+            umma_commit(acc_bar);
+        }
+    } else {
+        // ---------------- expansion: thread t writes weight row n0 + t of every stage
+        const int t = threadIdx.x - 64;
+        const int row = n0 + t;
+        const bool rv = row < W.rows;
+        const uint8_t *crow = W.codes + (int64_t)(rv ? row : 0) * W.code_row_bytes;
+        const __half *srow = W.scales + (int64_t)(rv ? row : 0) * W.scale_row_elems;
+        const uint8_t *cbl = sCB + (lane % CB::NREP) * CB::ENTRY;
+        const uint32_t swz = (uint32_t)(t & 7);
+
+        Blk cur, nxt;
+        __half sc_cur = __float2half(0.f), sc_nxt = __float2half(0.f);
+        if (rv) { cur.load(crow, 0); sc_cur = srow[0]; } else cur.zero();
+        for (int kb = 0; kb < nkb; kb++) {
+            if (kb + 1 < nkb) {
+                if (rv) { nxt.load(crow, kb + 1); sc_nxt = srow[kb + 1]; } else nxt.zero();
+            }
+            const int s = kb % STAGES, r = kb / STAGES;
+            const bool ok = r == 0 || mbar_wait(&empty[s], (r - 1) & 1);
+            if (__any_sync(0xffffffffu, !ok || *abort_flag)) {   // warp-uniform exit
+                if (lane == 0) flag_error(abort_flag);
+                break;
+            }
+            const uint32_t arow = smem_u32(sA + s * A_TILE_BYTES) + t * 128;
+            const __half2 s2 = __half2half2(sc_cur);
+            const float sf = __half2float(sc_cur);
+#pragma unroll
+            for (int c = 0; c < 8; c++) {
+                uint32_t o[4];
+                if constexpr (D == 2) {
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const uint32_t e = *reinterpret_cast<const uint32_t *>(cbl + cur.code(4 * c + j) * CB::STRIDE);
+                        o[j] = scale_pair<BF16T>(e, s2, sf);
+                    }
+                } else if constexpr (D == 4) {
+#pragma unroll
+                    for (int j = 0; j < 2; j++) {
+                        const uint2 e = *reinterpret_cast<const uint2 *>(cbl + cur.code(2 * c + j) * CB::STRIDE);
+                        o[2 * j] = scale_pair<BF16T>(e.x, s2, sf);
+                        o[2 * j + 1] = scale_pair<BF16T>(e.y, s2, sf);
+                    }
+                } else {
+                    const uint4 e = *reinterpret_cast<const uint4 *>(cbl + cur.code(c) * CB::STRIDE);
+                    o[0] = scale_pair<BF16T>(e.x, s2, sf);
+                    o[1] = scale_pair<BF16T>(e.y, s2, sf);
+                    o[2] = scale_pair<BF16T>(e.z, s2, sf);
+                    o[3] = scale_pair<BF16T>(e.w, s2, sf);
+                }
+                if (!rv) o[0] = o[1] = o[2] = o[3] = 0u;
+                sts128(arow + (((uint32_t)c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full_a[s]);
+            cur = nxt;
+            sc_cur = sc_nxt;
+        }
+
+        // ---------------- epilogue: TMEM -> registers -> y
+        __syncwarp();
+        const bool waited = mbar_wait(acc_bar, 0);
+        if (!waited) flag_error(abort_flag);
+        tc_fence_after();
+        if (__all_sync(0xffffffffu, waited && !*abort_flag)) {   // warp-uniform: tcgen05.ld is .sync.aligned
+            const int q = warp & 3;                  // TMEM lanes 32q..32q+31 belong to this warp
+            const int erow = n0 + q * 32 + lane;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BT; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+                tmem_ld_wait();
+                if (erow < W.rows) {
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        const int m = m0 + c0 + j;
+                        if (m < M) store_out(y, (int64_t)m * W.rows + erow, __uint_as_float(v[j]), yt);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// bf16 -> fp16 conversion of the activations (8 elements per thread).
+__global__ void bf16_to_f16_kernel(const __nv_bfloat16 *__restrict__ in, __half *__restrict__ out, int64_t n8)
+{
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    uint4 u = __ldg(reinterpret_cast<const uint4 *>(in) + i);
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[j]));
+        __half2 h = __floats2half2_rn(f.x, f.y);
+        w[j] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    reinterpret_cast<uint4 *>(out)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// Tensor map of activations [M][K] (16-bit, row stride K elements), box [BT][64], 128-B swizzle.
+static bool make_x_map(CUtensorMap *map, const void *x, bool bf16, int M, int K, int BT) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {GEMM_BK, (cuuint32_t)BT};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int BITS, int BT>
+static constexpr int gemm_stages() {
+    return SmemCB<D, BITS>::BYTES <= 32768 ? 4 : 3;
+}
+
+template <int D, int BITS, int BT, int STAGES>
+static constexpr size_t gemm_smem_bytes() {
+    return 1024 + (size_t)STAGES * (A_TILE_BYTES + BT * GEMM_BK * 2) + SmemCB<D, BITS>::BYTES +
+           (3 * STAGES + 1) * 8 + 16;
+}
+
+template <int D, int BITS, int BT, bool BF16T>
+static vq_status run_gemm_bt(const Mat &W, const void *x16, int M, void *y, int yt, cudaStream_t s)
+{
+    constexpr int STAGES = gemm_stages<D, BITS, BT>();
+    constexpr size_t smem = gemm_smem_bytes<D, BITS, BT, STAGES>();
+    static_assert(smem <= 232448, "shared memory budget");
+    CUtensorMap map;
+    if (!make_x_map(&map, x16, BF16T, M, W.cols, BT)) return VQ_ERR_CUDA;
+    auto kern = vq_gemm_kernel<D, BITS, BT, STAGES, BF16T>;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return VQ_ERR_CUDA;
+        attr = true;
+    }
+    dim3 grid((M + BT - 1) / BT, (W.rows + GEMM_BM - 1) / GEMM_BM);
+    kern<<<grid, GEMM_THREADS, smem, s>>>(map, W, M, y, yt);
+    VQ_CHECK_LAUNCH();
+    return VQ_OK;
+}
+
+template <int D, int BITS, bool BF16T>
+static vq_status run_gemm_geom(const Mat &W, const void *x16, int M, void *y, int yt, cudaStream_t s)
+{
+    if (M <= 32) return run_gemm_bt<D, BITS, 32, BF16T>(W, x16, M, y, yt, s);
+    if (M <= 64) return run_gemm_bt<D, BITS, 64, BF16T>(W, x16, M, y, yt, s);
+    if (M <= 128) return run_gemm_bt<D, BITS, 128, BF16T>(W, x16, M, y, yt, s);
+    return run_gemm_bt<D, BITS, 256, BF16T>(W, x16, M, y, yt, s);
+}
+
+template <bool BF16T>
+static vq_status run_gemm_tiles(const Mat &W, const void *x16, int M, void *y, int yt, cudaStream_t s)
+{
+    switch (geom_of(W.d, W.bits)) {
+    case G_D2_B8: return run_gemm_geom<2, 8, BF16T>(W, x16, M, y, yt, s);
+    case G_D4_B8: return run_gemm_geom<4, 8, BF16T>(W, x16, M, y, yt, s);
+    case G_D8_B8: return run_gemm_geom<8, 8, BF16T>(W, x16, M, y, yt, s);
+    case G_D2_B12: return run_gemm_geom<2, 12, BF16T>(W, x16, M, y, yt, s);
+    case G_D4_B12: return run_gemm_geom<4, 12, BF16T>(W, x16, M, y, yt, s);
+    case G_D8_B12: return run_gemm_geom<8, 12, BF16T>(W, x16, M, y, yt, s);
+    default: return VQ_ERR_UNSUPPORTED;
+    }
+}
+
+size_t gemm_workspace_bytes(const Mat &W, vq_dtype xt, int M, uint32_t flags)
+{
+    if (xt == VQ_BF16 && !(flags & VQ_GEMM_BF16_TILES)) return ((size_t)M * W.cols * 2 + 255) / 256 * 256;
+    return 0;
+}
+
+vq_status launch_gemm(const Mat &W, const void *x, vq_dtype xt, int M, void *y, vq_dtype yt, void *ws,
+                      size_t ws_bytes, uint32_t flags, cudaStream_t s)
+{
+    (void)ws_bytes;
+    if (flags & VQ_GEMM_BF16_TILES) return run_gemm_tiles<true>(W, x, M, y, (int)yt, s);
+    const void *x16 = x;
+    if (xt == VQ_BF16) {
+        const int64_t n8 = (int64_t)M * W.cols / 8;
+        bf16_to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const __nv_bfloat16 *)x, (__half *)ws, n8);
+        VQ_CHECK_LAUNCH();
+        x16 = ws;
+    }
+    return run_gemm_tiles<false>(W, x16, M, y, (int)yt, s);
+}
+
+vq_status read_device_error(cudaStream_t s, unsigned int *out)
+{
+    if (cudaStreamSynchronize(s) != cudaSuccess) return VQ_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(out, g_device_error, sizeof(unsigned int)) != cudaSuccess) return VQ_ERR_CUDA;
+    return VQ_OK;
+}
+
+}  // namespace vq
