@@ -38,7 +38,8 @@ def test_gemm_integer_exact(vqlib, d, bits, M):
     the exact integer product bit for bit (any misplaced tile element changes it)."""
     rng = np.random.default_rng(M * 7 + d + bits)
     rows, cols = 200, 512
-    Wi = rng.integers(-6, 7, (rows, cols)).astype(np.int64)
+    pool = rng.integers(-6, 7, (min(1 << bits, 200), d))          # <= K distinct subvectors
+    Wi = pool[rng.integers(0, pool.shape[0], (rows, cols // d))].reshape(rows, cols).astype(np.int64)
     xi = rng.integers(-8, 9, (M, cols)).astype(np.int64)
     data = encode_dense(Wi.astype(np.float32), d, bits)
     W = vqlib.VQMatrix.from_data(data)

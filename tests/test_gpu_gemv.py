@@ -78,3 +78,24 @@ def test_c2_mlp_decode_full(vqlib):
         y = run_gemv(vqlib, data, x, wl.F16)
         assert_out(y, ref)
         assert normwise(y.cpu().numpy(), ref) <= GEMV_F32_TOL
+
+
+@pytest.mark.parametrize("d,bits", GEOMS)
+@pytest.mark.parametrize("rows", [148, 301, 1000])
+@pytest.mark.parametrize("cols", [64, 1088, 2112, 17408])
+def test_gemv_row_streaming_path(vqlib, d, bits, rows, cols):
+    """Batch-1 shapes taken by the row-streaming kernel (rows >= number of SMs, scale rows
+    of whole 16-byte units): ragged row ranges per CTA, 1 to 272 units per row, partially
+    filled warps."""
+    data = wl.uniform_tensor(rows, cols, d, bits, seed=rows * 3 + cols + d * 5 + bits)
+    x = wl.activations(1, cols, seed=cols + 1, dtype=wl.F16)
+    ref = oracle.Tensor(data).linear(x, wl.F16)
+    assert_out(run_gemv(vqlib, data, x, wl.F16), ref)
+
+
+@pytest.mark.parametrize("xt", [wl.BF16, wl.F32])
+def test_gemv_row_streaming_other_dtypes(vqlib, xt):
+    data = wl.uniform_tensor(400, 1024, 8, 12, seed=31)
+    x = wl.activations(1, 1024, seed=32, dtype=xt)
+    ref = oracle.Tensor(data).linear(x, xt)
+    assert_out(run_gemv(vqlib, data, x, xt), ref)

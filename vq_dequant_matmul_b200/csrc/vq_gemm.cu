@@ -25,6 +25,7 @@
 #include <algorithm>
 
 #include "vq_codebook.cuh"
+#include "vq_gemm_api.cuh"
 #include "vq_internal.cuh"
 #include "vq_sm100.cuh"
 
@@ -101,16 +102,17 @@ __device__ __forceinline__ void flag_error(volatile int *abort_flag) {
     atomicExch(&g_device_error, 1u);
 }
 
+// One CTA: output tile rows [n0, n0 + 128) of expert e's matrix W against activation rows
+// [m0, m0 + mcount) of the tensor map; y[(m0 + j) * ldy + n] for j < mcount.
 template <int D, int BITS, int BT, int STAGES, bool BF16T>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, Mat W, int M, void *__restrict__ y, int yt)
+__device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, int e, int m0, int mcount,
+                                         int n0, void *__restrict__ y, int64_t ldy, int yt, uint8_t *smem_raw)
 {
     using CB = SmemCB<D, BITS>;
     using Blk = CodeBlock<D, BITS>;
     constexpr int B_TILE_BYTES = BT * GEMM_BK * 2;
     constexpr uint32_t TMEM_COLS = BT;          // fp32 accumulator: one column per token
 
-    extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = sA + STAGES * A_TILE_BYTES;
@@ -124,11 +126,11 @@ vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, Mat W, int M, void *__r
     volatile int *consumed = reinterpret_cast<volatile int *>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BT;
-    const int n0 = blockIdx.y * GEMM_BM;
     const int nkb = W.cols / GEMM_BK;
+    const uint8_t *codes_e = W.codes + (int64_t)e * W.expert_code_stride;
+    const __half *scales_e = W.scales + (int64_t)e * W.expert_scale_stride;
 
-    CB::stage(sCB, W.codebook);
+    CB::stage(sCB, W.codebook + (int64_t)e * W.expert_codebook_stride);
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
             mbar_init(&full_a[s], 4);
@@ -152,14 +154,14 @@ vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, Mat W, int M, void *__r
     if (warp == 0) {
         // ---------------- TMA producer: activation tiles
         if (lane == 0) {
-            tma_prefetch_map(&xmap);
+            tma_prefetch_map(xmap);
             int issued = 0;
             for (int kb = 0; kb < nkb; kb++) {
                 const int s = kb % STAGES, r = kb / STAGES;
                 if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1)) { flag_error(abort_flag); break; }
                 if (*abort_flag) break;
                 mbar_arrive_expect_tx(&full_b[s], B_TILE_BYTES);
-                tma_load_2d(sB + s * B_TILE_BYTES, &xmap, &full_b[s], kb * GEMM_BK, m0);
+                tma_load_2d(sB + s * B_TILE_BYTES, xmap, &full_b[s], kb * GEMM_BK, m0);
                 issued++;
             }
             // On an abort, wait (bounded) for the loads still in flight before leaving.
@@ -194,8 +196,8 @@ vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, Mat W, int M, void *__r
         const int t = threadIdx.x - 64;
         const int row = n0 + t;
         const bool rv = row < W.rows;
-        const uint8_t *crow = W.codes + (int64_t)(rv ? row : 0) * W.code_row_bytes;
-        const __half *srow = W.scales + (int64_t)(rv ? row : 0) * W.scale_row_elems;
+        const uint8_t *crow = codes_e + (int64_t)(rv ? row : 0) * W.code_row_bytes;
+        const __half *srow = scales_e + (int64_t)(rv ? row : 0) * W.scale_row_elems;
         const uint8_t *cbl = sCB + (lane % CB::NREP) * CB::ENTRY;
         const uint32_t swz = (uint32_t)(t & 7);
 
@@ -264,8 +266,8 @@ vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, Mat W, int M, void *__r
                 if (erow < W.rows) {
 #pragma unroll
                     for (int j = 0; j < 32; j++) {
-                        const int m = m0 + c0 + j;
-                        if (m < M) store_out(y, (int64_t)m * W.rows + erow, __uint_as_float(v[j]), yt);
+                        if (c0 + j < mcount)
+                            store_out(y, (int64_t)(m0 + c0 + j) * ldy + erow, __uint_as_float(v[j]), yt);
                     }
                 }
             }
@@ -277,6 +279,38 @@ vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, Mat W, int M, void *__r
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+
+template <int BT, int STAGES, bool BF16T>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ GemmArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const int z = blockIdx.z;
+    const Mat &W = a.W[z];
+    const int n0 = blockIdx.y * GEMM_BM;
+    if (n0 >= W.rows) return;                          // uniform over the CTA
+    int e = 0, m0, mcount;
+    if (a.t_exp) {
+        const int tile = blockIdx.x;
+        if (tile >= *a.ntiles) return;
+        e = a.t_exp[tile];
+        m0 = a.t_row[tile];
+        mcount = a.t_cnt[tile];
+    } else {
+        m0 = blockIdx.x * BT;
+        mcount = min(BT, a.M - m0);
+    }
+    switch (geom_of(W.d, W.bits)) {
+    case G_D2_B8: gemm_cta<2, 8, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D4_B8: gemm_cta<4, 8, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D8_B8: gemm_cta<8, 8, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D2_B12: gemm_cta<2, 12, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D4_B12: gemm_cta<4, 12, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D8_B12: gemm_cta<8, 12, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    default: break;
     }
 }
 
@@ -329,60 +363,75 @@ static bool make_x_map(CUtensorMap *map, const void *x, bool bf16, int M, int K,
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BITS, int BT>
-static constexpr int gemm_stages() {
-    return SmemCB<D, BITS>::BYTES <= 32768 ? 4 : 3;
+// Shared memory of a launch whose largest codebook table takes cb_bytes.
+static size_t gemm_smem_bytes(int BT, int stages, size_t cb_bytes) {
+    return 1024 + (size_t)stages * (A_TILE_BYTES + (size_t)BT * GEMM_BK * 2) + cb_bytes + (3 * stages + 1) * 8 + 16;
 }
 
-template <int D, int BITS, int BT, int STAGES>
-static constexpr size_t gemm_smem_bytes() {
-    return 1024 + (size_t)STAGES * (A_TILE_BYTES + BT * GEMM_BK * 2) + SmemCB<D, BITS>::BYTES +
-           (3 * STAGES + 1) * 8 + 16;
-}
-
-template <int D, int BITS, int BT, bool BF16T>
-static vq_status run_gemm_bt(const Mat &W, const void *x16, int M, void *y, int yt, cudaStream_t s)
-{
-    constexpr int STAGES = gemm_stages<D, BITS, BT>();
-    constexpr size_t smem = gemm_smem_bytes<D, BITS, BT, STAGES>();
-    static_assert(smem <= 232448, "shared memory budget");
-    CUtensorMap map;
-    if (!make_x_map(&map, x16, BF16T, M, W.cols, BT)) return VQ_ERR_CUDA;
-    auto kern = vq_gemm_kernel<D, BITS, BT, STAGES, BF16T>;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return VQ_ERR_CUDA;
-        attr = true;
+static size_t cb_table_bytes(const Mat &W) {
+    switch (geom_of(W.d, W.bits)) {
+    case G_D2_B8: return SmemCB<2, 8>::BYTES;
+    case G_D4_B8: return SmemCB<4, 8>::BYTES;
+    case G_D8_B8: return SmemCB<8, 8>::BYTES;
+    case G_D2_B12: return SmemCB<2, 12>::BYTES;
+    case G_D4_B12: return SmemCB<4, 12>::BYTES;
+    default: return SmemCB<8, 12>::BYTES;
     }
-    dim3 grid((M + BT - 1) / BT, (W.rows + GEMM_BM - 1) / GEMM_BM);
-    kern<<<grid, GEMM_THREADS, smem, s>>>(map, W, M, y, yt);
+}
+
+template <int BT, int STAGES, bool BF16T>
+static vq_status launch_gemm_cfg(const CUtensorMap &map, const GemmArgs &a, int nproj, int gx, size_t smem,
+                                 cudaStream_t s)
+{
+    auto kern = vq_gemm_kernel<BT, STAGES, BF16T>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return VQ_ERR_CUDA;
+    int rows = 0;
+    for (int z = 0; z < nproj; z++) rows = std::max(rows, a.W[z].rows);
+    dim3 grid(gx, (rows + GEMM_BM - 1) / GEMM_BM, nproj);
+    kern<<<grid, GEMM_THREADS, smem, s>>>(map, a);
     VQ_CHECK_LAUNCH();
     return VQ_OK;
 }
 
-template <int D, int BITS, bool BF16T>
-static vq_status run_gemm_geom(const Mat &W, const void *x16, int M, void *y, int yt, cudaStream_t s)
+template <int BT, bool BF16T>
+static vq_status launch_gemm_bt(const CUtensorMap &map, const GemmArgs &a, int nproj, int gx, cudaStream_t s)
 {
-    if (M <= 32) return run_gemm_bt<D, BITS, 32, BF16T>(W, x16, M, y, yt, s);
-    if (M <= 64) return run_gemm_bt<D, BITS, 64, BF16T>(W, x16, M, y, yt, s);
-    if (M <= 128) return run_gemm_bt<D, BITS, 128, BF16T>(W, x16, M, y, yt, s);
-    return run_gemm_bt<D, BITS, 256, BF16T>(W, x16, M, y, yt, s);
+    size_t cb = 0;
+    for (int z = 0; z < nproj; z++) cb = std::max(cb, cb_table_bytes(a.W[z]));
+    if (gemm_smem_bytes(BT, 4, cb) <= 232448)
+        return launch_gemm_cfg<BT, 4, BF16T>(map, a, nproj, gx, gemm_smem_bytes(BT, 4, cb), s);
+    if (gemm_smem_bytes(BT, 3, cb) <= 232448)
+        return launch_gemm_cfg<BT, 3, BF16T>(map, a, nproj, gx, gemm_smem_bytes(BT, 3, cb), s);
+    return VQ_ERR_UNSUPPORTED;
 }
 
-template <bool BF16T>
-static vq_status run_gemm_tiles(const Mat &W, const void *x16, int M, void *y, int yt, cudaStream_t s)
+// Run the GEMM over activation rows held in x16 ([rows][K] 16-bit, K = W.cols): dense
+// (a.t_exp == null, a.M rows) or grouped (tile list on the device, at most max_tiles).
+vq_status run_vq_gemm(const GemmArgs &a, int nproj, const void *x16, int x_rows, bool bf16, int BT,
+                      int max_tiles, cudaStream_t s)
 {
-    switch (geom_of(W.d, W.bits)) {
-    case G_D2_B8: return run_gemm_geom<2, 8, BF16T>(W, x16, M, y, yt, s);
-    case G_D4_B8: return run_gemm_geom<4, 8, BF16T>(W, x16, M, y, yt, s);
-    case G_D8_B8: return run_gemm_geom<8, 8, BF16T>(W, x16, M, y, yt, s);
-    case G_D2_B12: return run_gemm_geom<2, 12, BF16T>(W, x16, M, y, yt, s);
-    case G_D4_B12: return run_gemm_geom<4, 12, BF16T>(W, x16, M, y, yt, s);
-    case G_D8_B12: return run_gemm_geom<8, 12, BF16T>(W, x16, M, y, yt, s);
-    default: return VQ_ERR_UNSUPPORTED;
+    CUtensorMap map;
+    if (!make_x_map(&map, x16, bf16, x_rows, a.W[0].cols, BT)) return VQ_ERR_CUDA;
+    const int gx = a.t_exp ? max_tiles : (a.M + BT - 1) / BT;
+    if (gx < 1) return VQ_OK;
+    if (bf16) {
+        switch (BT) {
+        case 32: return launch_gemm_bt<32, true>(map, a, nproj, gx, s);
+        case 64: return launch_gemm_bt<64, true>(map, a, nproj, gx, s);
+        case 128: return launch_gemm_bt<128, true>(map, a, nproj, gx, s);
+        default: return launch_gemm_bt<256, true>(map, a, nproj, gx, s);
+        }
+    }
+    switch (BT) {
+    case 32: return launch_gemm_bt<32, false>(map, a, nproj, gx, s);
+    case 64: return launch_gemm_bt<64, false>(map, a, nproj, gx, s);
+    case 128: return launch_gemm_bt<128, false>(map, a, nproj, gx, s);
+    default: return launch_gemm_bt<256, false>(map, a, nproj, gx, s);
     }
 }
+
+static int dense_bt(int M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
 size_t gemm_workspace_bytes(const Mat &W, vq_dtype xt, int M, uint32_t flags)
 {
@@ -394,15 +443,35 @@ vq_status launch_gemm(const Mat &W, const void *x, vq_dtype xt, int M, void *y, 
                       size_t ws_bytes, uint32_t flags, cudaStream_t s)
 {
     (void)ws_bytes;
-    if (flags & VQ_GEMM_BF16_TILES) return run_gemm_tiles<true>(W, x, M, y, (int)yt, s);
+    GemmArgs a{};
+    a.W[0] = W;
+    a.y[0] = y;
+    a.ldy[0] = W.rows;
+    a.yt = (int)yt;
+    a.M = M;
+    const bool bf16_tiles = (flags & VQ_GEMM_BF16_TILES) != 0;
     const void *x16 = x;
-    if (xt == VQ_BF16) {
+    if (xt == VQ_BF16 && !bf16_tiles) {
         const int64_t n8 = (int64_t)M * W.cols / 8;
         bf16_to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const __nv_bfloat16 *)x, (__half *)ws, n8);
         VQ_CHECK_LAUNCH();
         x16 = ws;
     }
-    return run_gemm_tiles<false>(W, x16, M, y, (int)yt, s);
+    return run_vq_gemm(a, 1, x16, M, bf16_tiles, dense_bt(M), 0, s);
+}
+
+// Device address of the error word on the current device (looked up once per device).
+unsigned int *device_error_word()
+{
+    static unsigned int *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned int *>(p);
+    }
+    return addr[dev];
 }
 
 vq_status read_device_error(cudaStream_t s, unsigned int *out)

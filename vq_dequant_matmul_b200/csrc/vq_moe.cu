@@ -20,6 +20,7 @@
 #include <type_traits>
 
 #include "vq_codebook.cuh"
+#include "vq_gemm_api.cuh"
 #include "vq_gemv_body.cuh"
 #include "vq_internal.cuh"
 
@@ -260,6 +261,47 @@ __global__ void __launch_bounds__(GEMV_BODY_THREADS) moe_gemv_kernel(MoeGemvArgs
     }
 }
 
+// ------------------------------------------------------------------ prefill helpers
+
+// xg[pos] = fp16(x[token of the pair at pos]) for every valid pair (bucket order).
+template <typename XT>
+__global__ void moe_gather_kernel(const XT *__restrict__ x, const int *__restrict__ sorted, const int *__restrict__ offsets,
+                                  int E, int topk, int hidden, __half *__restrict__ xg)
+{
+    const int q = hidden / 8;
+    const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int total = offsets[E];
+    if (idx >= (int64_t)total * q) return;
+    const int j = (int)(idx / q), c = (int)(idx % q) * 8;
+    const int t = sorted[j] / topk;
+    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + (int64_t)t * hidden + c));
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    if constexpr (sizeof(XT) == 2 && !std::is_same<XT, __half>::value) {
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[k]));
+            __half2 h = __floats2half2_rn(f.x, f.y);
+            w[k] = *reinterpret_cast<uint32_t *>(&h);
+        }
+    }
+    *reinterpret_cast<uint4 *>(xg + (int64_t)j * hidden + c) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// h16 = fp16(silu(g) * u) for the valid rows.
+__global__ void moe_silu_mul_kernel(const float *__restrict__ g, const float *__restrict__ u,
+                                    const int *__restrict__ offsets, int E, int inter, __half *__restrict__ h)
+{
+    const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t n4 = (int64_t)offsets[E] * inter / 4;
+    if (idx >= n4) return;
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(g) + idx);
+    const float4 b = __ldg(reinterpret_cast<const float4 *>(u) + idx);
+    const __half2 lo = __floats2half2_rn(a.x / (1.f + expf(-a.x)) * b.x, a.y / (1.f + expf(-a.y)) * b.y);
+    const __half2 hi = __floats2half2_rn(a.z / (1.f + expf(-a.z)) * b.z, a.w / (1.f + expf(-a.w)) * b.w);
+    reinterpret_cast<__half2 *>(h)[2 * idx] = lo;
+    reinterpret_cast<__half2 *>(h)[2 * idx + 1] = hi;
+}
+
 // ------------------------------------------------------------------ 4. combine
 
 __global__ void moe_combine_kernel(const float *__restrict__ o, const int *__restrict__ pos,
@@ -288,6 +330,7 @@ __global__ void moe_combine_kernel(const float *__restrict__ o, const int *__res
 }
 
 // ------------------------------------------------------------------ host
+
 
 static size_t cb_smem_bytes(const Mat &W) {
     switch (geom_of(W.d, W.bits)) {
@@ -339,8 +382,13 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     auto I = [&](size_t off) { return reinterpret_cast<int *>(W8 + off); };
     auto F = [&](size_t off) { return reinterpret_cast<float *>(W8 + off); };
 
+    // Tensor cores once experts see several tokens on average; the grouped GEMV otherwise.
+    const double per_expert = (double)L.P / std::min(E, L.P);
+    const bool use_gemm = per_expert >= 4.0;
+    const int BT = per_expert <= 24 ? 32 : per_expert <= 48 ? 64 : 128;
+
     BucketArgs b;
-    b.ids = ids; b.P = L.P; b.E = E; b.BT = 32;
+    b.ids = ids; b.P = L.P; b.E = E; b.BT = BT;
     b.status = reinterpret_cast<unsigned int *>(W8 + L.status);
     b.counts = I(L.counts); b.offsets = I(L.offsets); b.sorted = I(L.sorted); b.pos = I(L.pos);
     b.act = I(L.act); b.nact = I(L.nact); b.t_exp = I(L.t_exp); b.t_row = I(L.t_row); b.t_cnt = I(L.t_cnt);
@@ -353,13 +401,44 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     VQ_CHECK_LAUNCH();
 
     const int max_active = std::min(E, L.P);
+    vq_status st;
+    if (use_gemm) {
+        __half *xg = reinterpret_cast<__half *>(W8 + L.xg);
+        __half *h16 = reinterpret_cast<__half *>(W8 + L.h16);
+        const int64_t ng = (int64_t)L.P * (hidden / 8);
+        if (xt == VQ_F16)
+            moe_gather_kernel<__half><<<(unsigned)((ng + 255) / 256), 256, 0, s>>>((const __half *)x, b.sorted, b.offsets, E, topk, hidden, xg);
+        else
+            moe_gather_kernel<__nv_bfloat16><<<(unsigned)((ng + 255) / 256), 256, 0, s>>>((const __nv_bfloat16 *)x, b.sorted, b.offsets, E, topk, hidden, xg);
+        VQ_CHECK_LAUNCH();
+        const int max_tiles = std::min(L.max_tiles, (L.P + BT - 1) / BT + E);
+        GemmArgs ga{};
+        ga.W[0] = gate; ga.W[1] = up;
+        ga.y[0] = F(L.g); ga.y[1] = F(L.u);
+        ga.ldy[0] = ga.ldy[1] = inter;
+        ga.yt = VQ_F32;
+        ga.t_exp = b.t_exp; ga.t_row = b.t_row; ga.t_cnt = b.t_cnt; ga.ntiles = b.ntiles;
+        if ((st = run_vq_gemm(ga, 2, xg, L.P, false, BT, max_tiles, s)) != VQ_OK) return st;
+        const int64_t nh = (int64_t)L.P * inter / 4;
+        moe_silu_mul_kernel<<<(unsigned)((nh + 255) / 256), 256, 0, s>>>(F(L.g), F(L.u), b.offsets, E, inter, h16);
+        VQ_CHECK_LAUNCH();
+        GemmArgs gd = ga;
+        gd.W[0] = down;
+        gd.y[0] = F(L.o);
+        gd.ldy[0] = hidden;
+        if ((st = run_vq_gemm(gd, 1, h16, L.P, false, BT, max_tiles, s)) != VQ_OK) return st;
+        const int64_t n = (int64_t)T * (hidden / 4);
+        moe_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(F(L.o), b.pos, w, T, topk, hidden, y, (int)yt);
+        VQ_CHECK_LAUNCH();
+        return VQ_OK;
+    }
     MoeGemvArgs a{};
     a.sorted = b.sorted; a.offsets = b.offsets; a.act = b.act; a.nact = b.nact; a.topk = topk;
     // gate and up in one grouped launch
     a.W[0] = gate; a.W[1] = up;
     a.out[0] = F(L.g); a.out[1] = F(L.u);
     a.x = x;
-    vq_status st = xt == VQ_F16 ? launch_moe_gemv<0>(a, 2, max_active, s) : launch_moe_gemv<1>(a, 2, max_active, s);
+    st = xt == VQ_F16 ? launch_moe_gemv<0>(a, 2, max_active, s) : launch_moe_gemv<1>(a, 2, max_active, s);
     if (st != VQ_OK) return st;
     // down, input silu(g) * u
     a.W[0] = down;
