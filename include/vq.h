@@ -156,6 +156,27 @@ vq_status vq_moe_grouped(const vq_matrix *gate, const vq_matrix *up, const vq_ma
                          const float *expert_w, int32_t topk, void *y, vq_dtype yt,
                          void *ws, size_t ws_bytes, vq_stream_t stream);
 
+/* vq_moe_grouped for callers that cannot allocate device memory (for example code that
+ * runs where cudaMalloc is not allowed, or a caller without its own device allocator):
+ * same arguments and results as vq_moe_grouped, minus the workspace.  There is no
+ * counterpart on the pages; this is a convenience of this library.
+ *   - The scratch is a fixed 16 MiB array inside the library's device image; every GPU
+ *     that loads the library holds it until the process exits.  Calls whose
+ *     vq_moe_workspace_size exceeds 16 MiB (about T * topk * (10 * inter + 6 * hidden)
+ *     bytes plus small tables: decode-sized batches) return VQ_ERR_WORKSPACE and launch
+ *     nothing.
+ *   - The first call on each device looks up the array's device address (with that
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents (every call
+ *     rewrites all it reads).  Calls that overlap on the GPU race on it: serialise them.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - Bad expert ids are skipped as in vq_moe_grouped; their count stays in the shared
+ *     scratch and is not reported by vq_read_device_status. */
+vq_status vq_moe_grouped_noalloc(const vq_matrix *gate, const vq_matrix *up, const vq_matrix *down,
+                                 const void *x, vq_dtype xt, int32_t T, const int32_t *expert_ids,
+                                 const float *expert_w, int32_t topk, void *y, vq_dtype yt,
+                                 vq_stream_t stream);
+
 /* Synchronise `stream`, then report what the device recorded: VQ_ERR_TIMEOUT if any
  * kernel of this library gave up a bounded wait since the library was loaded (a bug
  * signal; the kernel ended instead of hanging), else, when ws is not NULL, the status

@@ -56,6 +56,7 @@ _SIGS = {
     "vq_gemm_workspace_size": (_I32, [_M, _I32, _I32, ctypes.c_uint32, ctypes.POINTER(_SZ)]),
     "vq_moe_workspace_size": (_I32, [_I32, _I32, _I32, _I32, _I32, ctypes.POINTER(_SZ)]),
     "vq_moe_grouped": (_I32, [_M, _M, _M, _P, _I32, _I32, _P, _P, _I32, _P, _I32, _P, _SZ, _P]),
+    "vq_moe_grouped_noalloc": (_I32, [_M, _M, _M, _P, _I32, _I32, _P, _P, _I32, _P, _I32, _P]),
     "vq_read_device_status": (_I32, [_P, _P]),
     "vq_status_string": (ctypes.c_char_p, [_I32]),
     "vq_version": (ctypes.c_char_p, []),
@@ -217,6 +218,16 @@ def vq_moe_grouped(gate: VQMatrix, up: VQMatrix, down: VQMatrix, x: torch.Tensor
     _check(_lib.vq_moe_grouped(gate.ptr, up.ptr, down.ptr, _ptr(x), _TORCH_TO_VQ[x.dtype], T,
                                _ptr(expert_ids), _ptr(expert_w), topk, _ptr(y), _TORCH_TO_VQ[y.dtype],
                                _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "vq_moe_grouped")
+
+
+def vq_moe_grouped_noalloc(gate: VQMatrix, up: VQMatrix, down: VQMatrix, x: torch.Tensor,
+                           expert_ids: torch.Tensor, expert_w: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """vq_moe_grouped without a workspace: for callers that cannot allocate device memory.
+    Uses the library's fixed 16 MiB device scratch (decode-sized batches only)."""
+    T, topk = expert_ids.shape
+    _check(_lib.vq_moe_grouped_noalloc(gate.ptr, up.ptr, down.ptr, _ptr(x), _TORCH_TO_VQ[x.dtype], T,
+                                       _ptr(expert_ids), _ptr(expert_w), topk, _ptr(y), _TORCH_TO_VQ[y.dtype],
+                                       _stream(stream)), "vq_moe_grouped_noalloc")
 
 
 def vq_read_device_status(ws: torch.Tensor, stream=None) -> int:

@@ -19,6 +19,8 @@ vq_status launch_moe(const Mat &, const Mat &, const Mat &, const void *, vq_dty
                      cudaStream_t);
 vq_status read_moe_status(const void *, cudaStream_t);
 vq_status read_device_error(cudaStream_t, unsigned int *);
+size_t moe_static_scratch_bytes();
+void *moe_static_scratch();
 }  // namespace vq
 
 namespace {
@@ -162,6 +164,24 @@ vq_status vq_moe_grouped(const vq_matrix *gate, const vq_matrix *up, const vq_ma
     if (ws_bytes < need) return VQ_ERR_WORKSPACE;
     return vq::launch_moe(vq::to_mat(*gate), vq::to_mat(*up), vq::to_mat(*down), x, xt, T, expert_ids,
                           expert_w, topk, y, yt, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+vq_status vq_moe_grouped_noalloc(const vq_matrix *gate, const vq_matrix *up, const vq_matrix *down,
+                                 const void *x, vq_dtype xt, int32_t T, const int32_t *expert_ids,
+                                 const float *expert_w, int32_t topk, void *y, vq_dtype yt, vq_stream_t stream)
+{
+    vq_status st;
+    if ((st = check_matrix(gate)) != VQ_OK || (st = check_matrix(up)) != VQ_OK ||
+        (st = check_matrix(down)) != VQ_OK)
+        return st;
+    size_t need = 0;
+    if ((st = vq_moe_workspace_size(T, topk, gate->num_experts, gate->cols, gate->rows, &need)) != VQ_OK)
+        return st;
+    if (need > vq::moe_static_scratch_bytes()) return VQ_ERR_WORKSPACE;
+    void *scratch = vq::moe_static_scratch();
+    if (!scratch) return VQ_ERR_CUDA;
+    return vq_moe_grouped(gate, up, down, x, xt, T, expert_ids, expert_w, topk, y, yt, scratch,
+                          vq::moe_static_scratch_bytes(), stream);
 }
 
 vq_status vq_read_device_status(const void *ws, vq_stream_t stream)

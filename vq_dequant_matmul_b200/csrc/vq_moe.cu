@@ -460,4 +460,29 @@ vq_status read_moe_status(const void *ws, cudaStream_t s)
     return bad ? VQ_ERR_DEVICE_FLAG : VQ_OK;
 }
 
+// ------------------------------------------------------------------ allocation-free variant
+
+// Scratch of the allocation-free entry point (vq_moe_grouped_noalloc): a fixed array in
+// the library's device image, present on every GPU that loads the library until exit.
+constexpr size_t MOE_STATIC_SCRATCH_BYTES = (size_t)16 << 20;
+static __device__ __align__(256) unsigned char g_moe_static_scratch[MOE_STATIC_SCRATCH_BYTES];
+
+size_t moe_static_scratch_bytes() { return MOE_STATIC_SCRATCH_BYTES; }
+
+// Device address of the static scratch on the current device.  Host code cannot use the
+// array's name as a device address, so the address is looked up once per device (with
+// that device current) and cached.  Returns nullptr if the lookup fails.
+void *moe_static_scratch()
+{
+    static void *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_moe_static_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace vq
