@@ -1,18 +1,26 @@
 #!/usr/bin/env python
 """Benchmark of the VQ dequantize-and-multiply hot path on B200.
 
-Workload (one "step"): the dense MLP trio at d2/K256 with k-means codebooks (gate and
-up [17408][5120], down [5120][17408]): one decode token through the trio (three GEMV
-launches, fp16 activations, fp32 outputs) and one 2048-token bf16 prefill through the
-trio (three tensor-core GEMM launches).  Inputs are synthetic and seeded (workloads
-package); three copies of the trio (3 x 142 MB) are rotated so that no step finds its
-weights in the 126 MB L2.
+One step = the whole hot path of the dense MLP trio at d2/K256 with k-means codebooks
+(gate and up [17408][5120], down [5120][17408]):
+  * decode: one token through the trio (three GEMV launches, fp16 activations, fp32
+    outputs);
+  * prefill: 2048 bf16 tokens through the trio (three tensor-core GEMM launches, bf16
+    outputs; the bf16 activations are converted to fp16 inside vq_gemm).
+Three copies of the trio (3 x 142 MB) rotate, so no step finds its weights in the 126 MB
+L2.  The MoE layers (256 experts top-8 with mixed tiers; 512 experts top-10) are timed
+as extra legs of the same run, with L2 flushed between iterations.
+
+`value` is the decode GEMV's effective HBM bandwidth (algorithmic bytes: packed codes +
+scales + codebook + x + y, over the decode launches' device time); `prefill` holds the
+prefill TFLOP/s; `moe` the MoE layers' tokens/s.  Inputs are synthetic and seeded
+(workloads package).
 
 `python bench.py [--gpus N] [--steps K] [--warmup W]` prints one JSON line.  With N > 1
-(torchrun) every rank runs an independent replica (the path has no exchange step) and the
-line reports the whole-job throughput over the max-over-ranks device time.
-`--impl reference` times the CPU oracle on the host cores instead (a bounded sample of the
-same workload per step).
+(torchrun) every rank runs an independent replica (the path has no exchange step) and
+the line reports whole-job throughput over the max-over-ranks device time.
+`--impl reference` times the CPU oracle on the host cores instead (a bounded sample of
+the same workload per step).
 """
 from __future__ import annotations
 
@@ -35,6 +43,7 @@ import workloads as wl  # noqa: E402
 METRIC = "VQ GEMV effective HBM GB/s (% of peak); prefill TFLOP/s; MoE layer tokens/s"
 PREFILL_TOKENS = 2048
 COPIES = 3
+L2_FLUSH_BYTES = 256 << 20
 
 
 def peaks():
@@ -108,13 +117,27 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# ----------------------------------------------------------------------------- workload bytes
+# ----------------------------------------------------------------------------- algorithmic sizes
+
+def weight_bytes(data, experts=1):
+    """Packed codes + fp16 scales (+ one codebook) of a tensor."""
+    rb = ((data.cols // data.d + 31) // 32) * 4 * data.bits
+    return experts * (data.rows * rb + data.rows * (data.cols // 64) * 2) + (1 << data.bits) * data.d * 2
+
 
 def gemv_bytes(data, x_el=2, y_el=4, batch=1):
     """Algorithmic bytes of one GEMV: packed codes + scales + codebook + x + y."""
-    rb = ((data.cols // data.d + 31) // 32) * 4 * data.bits
-    return (data.rows * rb + data.rows * (data.cols // 64) * 2 + (1 << data.bits) * data.d * 2
-            + batch * data.cols * x_el + batch * data.rows * y_el)
+    return weight_bytes(data) + batch * data.cols * x_el + batch * data.rows * y_el
+
+
+def gemm_flops(data, M):
+    return 2.0 * M * data.rows * data.cols
+
+
+def _dev_bits(a, dev, dtype):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(dtype)
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -127,100 +150,186 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     pk = peaks()
+    stream = torch.cuda.current_stream()
 
     trio = wl.c2_mlp_tensors(device=str(dev))
     mats = [[vq.VQMatrix.from_data(t, device=dev) for t in trio]]
     for _ in range(COPIES - 1):
         mats.append([vq.VQMatrix(m.codebook.clone(), m.codes.clone(), m.scales.clone(), m.rows, m.cols,
                                  m.d, m.bits) for m in mats[0]])
-    xd = [torch.from_numpy(wl.activations(1, t.cols, wl.BASE_SEED + 10 + i, wl.F16).view(np.int16))
-          .to(dev).view(torch.float16) for i, t in enumerate(trio)]
+    # decode inputs / outputs
+    xd = [_dev_bits(wl.activations(1, t.cols, wl.BASE_SEED + 10 + i, wl.F16), dev, torch.float16)
+          for i, t in enumerate(trio)]
     yd = [torch.empty((1, t.rows), dtype=torch.float32, device=dev) for t in trio]
-    dec_bytes = [gemv_bytes(t) for t in trio]
-    step_bytes = sum(dec_bytes)
-    stream = torch.cuda.current_stream()
+    # prefill inputs / outputs (bf16 activations and outputs)
+    M = PREFILL_TOKENS
+    xp = [_dev_bits(wl.activations(M, t.cols, wl.BASE_SEED + 20 + i, wl.BF16), dev, torch.bfloat16)
+          for i, t in enumerate(trio)]
+    yp = [torch.empty((M, t.rows), dtype=torch.bfloat16, device=dev) for t in trio]
+    ws_bytes = max(vq.vq_gemm_workspace_size(mats[0][i], torch.bfloat16, M) for i in range(3))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
 
-    def decode(c, ev=None):
+    dec_bytes = [gemv_bytes(t) for t in trio]
+    pre_flops = [gemm_flops(t, M) for t in trio]
+
+    def step(c, ev=None):
         for i in range(3):
             if ev is not None:
                 ev[i][0].record(stream)
             vq.vq_gemv(mats[c][i], xd[i], yd[i])
             if ev is not None:
                 ev[i][1].record(stream)
+        for i in range(3):
+            if ev is not None:
+                ev[3 + i][0].record(stream)
+            vq.vq_gemm(mats[c][i], xp[i], yp[i], ws)
+            if ev is not None:
+                ev[3 + i][1].record(stream)
 
-    # warm-up
     for s in range(args.warmup):
-        decode(s % COPIES)
+        step(s % COPIES)
     torch.cuda.synchronize()
 
-    # timed region: K steps, per-launch events on the launching stream
     K = args.steps
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)] for _ in range(K)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(6)] for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         start.record(stream)
         for s in range(K):
-            decode(s % COPIES, evs[s])
+            step(s % COPIES, evs[s])
         stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    total_ms = start.elapsed_time(stop)
-    kern_ms = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(K)) for i in range(3)]
-    total_ms = max_over_ranks(total_ms, world)
-    ms_per_step = total_ms / K
-    value = step_bytes * K * world / (total_ms * 1e-3) / 1e9
+    total_ms = max_over_ranks(start.elapsed_time(stop), world)
+    kern_ms = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(K)) / K for i in range(6)]
+    dec_ms = max_over_ranks(sum(kern_ms[:3]), world)
+    pre_ms = max_over_ranks(sum(kern_ms[3:]), world)
+    value = sum(dec_bytes) * world / (dec_ms * 1e-3) / 1e9
+    prefill_tflops = sum(pre_flops) * world / (pre_ms * 1e-3) / 1e12
 
-    gemv_ms = sum(kern_ms) / (3 * K)
-    gemv_gbs = step_bytes / 3 / (gemv_ms * 1e-3) / 1e9
-    roofline = {"kernel": "gemv_b1_kernel<2,8,half>", "bound": "hbm", "achieved": round(gemv_gbs, 1),
+    gemv_gbs = sum(dec_bytes) / (sum(kern_ms[:3]) * 1e-3) / 1e9
+    roofline = {"kernel": "gemv_stream_kernel<2,8,half>", "bound": "hbm", "achieved": round(gemv_gbs, 1),
                 "peak": pk["hbm"], "unit": "GB/s", "frac": round(gemv_gbs / pk["hbm"], 4),
-                "traffic": args.traffic, "peak_source": pk["source"],
-                "per_projection_gbs": [round(dec_bytes[i] / (kern_ms[i] / K * 1e-3) / 1e9, 1) for i in range(3)]}
+                "traffic": args.traffic, "peak_source": pk["source"] + " (burst copy)",
+                "per_projection_gbs": [round(dec_bytes[i] / (kern_ms[i] * 1e-3) / 1e9, 1) for i in range(3)],
+                "frac_of_nominal_8tbs": round(gemv_gbs / 8000.0, 4)}
+    gemm_tf = sum(pre_flops) / (sum(kern_ms[3:]) * 1e-3) / 1e12
+    prefill = {"value": round(prefill_tflops, 1), "unit": "TFLOP/s", "ms": round(pre_ms, 4),
+               "tokens": M, "flops": sum(pre_flops),
+               "roofline": {"kernel": "vq_gemm_kernel (tcgen05, fp16 tiles)", "bound": "tensor",
+                            "achieved": round(gemm_tf, 1), "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                            "frac": round(gemm_tf / pk["bf16_sus"], 4),
+                            "frac_of_burst_peak": round(gemm_tf / pk["bf16"], 4),
+                            "peak_source": pk["source"] + " (sustained bf16 cuBLAS; fp16 has the same rate)",
+                            "traffic": None,
+                            "per_projection_tflops": [round(pre_flops[i] / (kern_ms[3 + i] * 1e-3) / 1e12, 1)
+                                                      for i in range(3)]}}
 
-    # end to end through the C ABI: pinned host x -> device, GEMVs, device y -> pinned host
-    xh = [x.cpu().pin_memory() for x in xd]
-    yh = [torch.empty_like(y, device="cpu").pin_memory() for y in yd]
+    # end to end through the C ABI: pinned host inputs -> device, step, outputs -> pinned host
+    xh = [x.cpu().pin_memory() for x in xd + xp]
+    yh = [torch.empty_like(y, device="cpu").pin_memory() for y in yd + yp]
+    xdev, ydev = xd + xp, yd + yp
     h2d = sum(x.numel() * x.element_size() for x in xh)
     d2h = sum(y.numel() * y.element_size() for y in yh)
-    for s in range(args.warmup):
-        for i in range(3):
-            xd[i].copy_(xh[i], non_blocking=True)
-        decode(s % COPIES)
-        for i in range(3):
-            yh[i].copy_(yd[i], non_blocking=True)
+    K2 = max(3, min(K, args.e2e_steps))
+
+    def e2e_step(c):
+        for i in range(6):
+            xdev[i].copy_(xh[i], non_blocking=True)
+        step(c)
+        for i in range(6):
+            yh[i].copy_(ydev[i], non_blocking=True)
+
+    for s in range(3):
+        e2e_step(s % COPIES)
     torch.cuda.synchronize()
     barrier(world)
     start.record(stream)
-    for s in range(K):
-        for i in range(3):
-            xd[i].copy_(xh[i], non_blocking=True)
-        decode(s % COPIES)
-        for i in range(3):
-            yh[i].copy_(yd[i], non_blocking=True)
+    for s in range(K2):
+        e2e_step(s % COPIES)
     stop.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(start.elapsed_time(stop), world)
-    e2e = {"value": round(step_bytes * K * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)}
+    e2e_ms = max_over_ranks(start.elapsed_time(stop), world) / K2
+    e2e = {"value": round(sum(dec_bytes) * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+           "steps": K2,
+           "note": "decode bytes over the whole end-to-end step (decode + 2048-token prefill + copies)"}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": "dense MLP trio d2/K256 (gate/up 17408x5120, down 5120x17408), "
-                               "batch-1 decode through the trio",
-                   "weights_bytes_per_step": step_bytes, "l2": f"{COPIES} weight copies rotated (> L2)",
+        "config": {"workload": "dense MLP trio d2/K256 k-means codebooks (gate/up 17408x5120, down "
+                               "5120x17408): batch-1 fp16 decode + 2048-token bf16 prefill per step",
+                   "decode_bytes_per_step": sum(dec_bytes), "prefill_flops_per_step": sum(pre_flops),
+                   "l2": f"{COPIES} weight copies rotated (3 x 142 MB > 126 MB L2)",
                    "parallelism": f"replicas{world}"},
-        "frac_of_nominal_8tbs": round(value / 8000.0, 4),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": 3 * K,
+        "roofline": roofline, "prefill": prefill, "e2e": e2e,
+        "clocks": clk.summary(),
     }
-    clocks = clk.summary()
-    line["clocks"] = clocks
+    # timed region: per step 3 GEMV launches + 3 x (bf16->fp16 conversion + GEMM)
+    line["gpu_launches"] = 9 * K
+    if not args.no_moe:
+        line["moe"] = moe_legs(args, vq, dev, pk, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_decode(trio, args.cpu_rows)
+        line["cpu_baseline"] = cpu_baseline(trio, args.cpu_rows)
     return line
+
+
+def moe_legs(args, vq, dev, pk, world):
+    """Routed MoE layers: tokens/s per (layer, T), L2 flushed between timed iterations."""
+    import torch
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, builder, Ts in (("c4_256x_top8_mixed", wl.c4_moe, (1, 16, 512)),
+                              ("c5_512x_top10_d4k256", wl.c5_moe_large, (1, 1024))):
+        mw = builder()
+        G, U, D = (vq.VQMatrix.from_data(t, device=dev) for t in (mw.gate, mw.up, mw.down))
+        per_expert = sum(weight_bytes(t) - (1 << t.bits) * t.d * 2 for t in (mw.gate, mw.up, mw.down))
+        cbs = sum((1 << t.bits) * t.d * 2 for t in (mw.gate, mw.up, mw.down))
+        for T in Ts:
+            nrep = 8
+            inputs = []
+            for r in range(nrep):
+                x, ids, w = wl.moe_inputs(mw, T, seed=wl.BASE_SEED + 300 + 17 * r + T)
+                inputs.append((_dev_bits(x, dev, torch.float16), torch.from_numpy(ids).to(dev),
+                               torch.from_numpy(w).to(dev), len(np.unique(ids))))
+            y = torch.empty((T, mw.hidden), dtype=torch.float32, device=dev)
+            ws = torch.empty(vq.vq_moe_workspace_size(T, mw.topk, mw.E, mw.hidden, mw.inter),
+                             dtype=torch.uint8, device=dev)
+            for r in range(3):
+                xdv, idd, wd, _ = inputs[r % nrep]
+                vq.vq_moe_grouped(G, U, D, xdv, idd, wd, y, ws)
+            torch.cuda.synchronize()
+            iters = args.moe_iters
+            times, nbytes = [], []
+            for it in range(iters):
+                xdv, idd, wd, ne = inputs[it % nrep]
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                vq.vq_moe_grouped(G, U, D, xdv, idd, wd, y, ws)
+                e1.record(stream)
+                times.append((e0, e1))
+                nbytes.append(ne * per_expert + cbs + T * mw.hidden * 2 * 2)
+            torch.cuda.synchronize()
+            ms = [a.elapsed_time(b) for a, b in times]
+            mean_ms = max_over_ranks(sum(ms) / len(ms), world)
+            gbs = sum(nbytes) / len(nbytes) / (mean_ms * 1e-3) / 1e9
+            out[f"{name}_T{T}"] = {"tokens_per_s": round(T * world / (mean_ms * 1e-3), 1), "ms": round(mean_ms, 4),
+                                   "effective_gbs": round(gbs, 1), "hbm_frac": round(gbs / pk["hbm"], 4),
+                                   "path": "grouped tcgen05 GEMM" if T * mw.topk / min(mw.E, T * mw.topk) >= 4
+                                   else "grouped GEMV", "iters": iters, "l2": "flushed between iterations"}
+            out[f"{name}_T{T}"]["gpu_launches"] = iters * (6 if out[f"{name}_T{T}"]["path"].startswith("grouped tc")
+                                                            else 4)
+            del ws, y
+        del G, U, D, mw
+        torch.cuda.empty_cache()
+    return out
 
 
 def barrier(world):
@@ -243,26 +352,31 @@ def max_over_ranks(v, world):
 
 # ----------------------------------------------------------------------------- oracle arm
 
-def cpu_baseline_decode(trio, rows_per_proj):
-    """The oracle (as it stands) on a bounded sample: the first `rows_per_proj` rows of
-    each projection of the decode step, compute only (packing is input preparation).
-    Reported in the same unit (effective GB/s)."""
+def _oracle_sample(trio, rows):
     import oracle
 
-    t_all, nbytes = 0.0, 0
+    subs = []
     for i, t in enumerate(trio):
-        sub = wl.VQTensorData(min(rows_per_proj, t.rows), t.cols, t.d, t.bits, t.codebook,
-                              t.codes[:, :rows_per_proj], t.scales[:, :rows_per_proj])
-        ot = oracle.Tensor(sub)
-        x = wl.activations(1, t.cols, wl.BASE_SEED + 10 + i, wl.F16)
-        t1 = time.perf_counter()
+        sub = wl.VQTensorData(min(rows, t.rows), t.cols, t.d, t.bits, t.codebook,
+                              t.codes[:, :rows], t.scales[:, :rows])
+        subs.append((oracle.Tensor(sub), gemv_bytes(sub), wl.activations(1, t.cols, wl.BASE_SEED + 10 + i, wl.F16)))
+    return subs
+
+
+def cpu_baseline(trio, rows):
+    """The oracle (as it stands) on a bounded sample: the first `rows` rows of each
+    projection of the decode step, compute only.  Same unit (effective GB/s)."""
+    import oracle
+
+    subs = _oracle_sample(trio, rows)
+    t1 = time.perf_counter()
+    for ot, _, x in subs:
         ot.linear(x, wl.F16)
-        t_all += time.perf_counter() - t1
-        nbytes += gemv_bytes(sub)
-    return {"value": round(nbytes / t_all / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"first {rows_per_proj} rows of each of gate/up/down, batch-1 decode "
-                      f"({nbytes} algorithmic bytes), {t_all:.2f} s"}
+    dt = time.perf_counter() - t1
+    nbytes = sum(b for _, b, _ in subs)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {rows} rows of each of gate/up/down, batch-1 decode ({nbytes} algorithmic bytes), "
+                      f"{dt:.2f} s"}
 
 
 def run_reference(args, rank, world):
@@ -272,24 +386,18 @@ def run_reference(args, rank, world):
     import oracle
 
     trio = wl.c2_mlp_tensors(device="cuda" if _cuda() else "cpu")
-    rows = args.cpu_rows
-    subs, xs = [], []
-    for i, t in enumerate(trio):
-        sub = wl.VQTensorData(min(rows, t.rows), t.cols, t.d, t.bits, t.codebook,
-                              t.codes[:, :rows], t.scales[:, :rows])
-        subs.append((oracle.Tensor(sub), gemv_bytes(sub)))
-        xs.append(wl.activations(1, t.cols, wl.BASE_SEED + 10 + i, wl.F16))
-    nbytes = sum(b for _, b in subs)
+    subs = _oracle_sample(trio, args.cpu_rows)
+    nbytes = sum(b for _, b, _ in subs)
     for _ in range(args.warmup):
-        for (ot, _), x in zip(subs, xs):
+        for ot, _, x in subs:
             ot.linear(x, wl.F16)
     t1 = time.perf_counter()
     for _ in range(args.steps):
-        for (ot, _), x in zip(subs, xs):
+        for ot, _, x in subs:
             ot.linear(x, wl.F16)
     dt = time.perf_counter() - t1
     v = nbytes * args.steps / dt / 1e9
-    sample = f"first {rows} rows of each of gate/up/down, batch-1 decode ({nbytes} bytes per step)"
+    sample = f"first {args.cpu_rows} rows of each of gate/up/down, batch-1 decode ({nbytes} bytes per step)"
     return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -312,13 +420,16 @@ def _cuda():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--moe-iters", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-moe", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+                    help="dram bytes per launch of the decode GEMV from an ncu capture")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

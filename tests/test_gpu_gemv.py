@@ -81,20 +81,21 @@ def test_c2_mlp_decode_full(vqlib):
 
 
 @pytest.mark.parametrize("d,bits", GEOMS)
-@pytest.mark.parametrize("rows", [148, 301, 1000])
-@pytest.mark.parametrize("cols", [64, 1088, 2112, 17408])
-def test_gemv_row_streaming_path(vqlib, d, bits, rows, cols):
-    """Batch-1 shapes taken by the row-streaming kernel (rows >= number of SMs, scale rows
-    of whole 16-byte units): ragged row ranges per CTA, 1 to 272 units per row, partially
-    filled warps."""
-    data = wl.uniform_tensor(rows, cols, d, bits, seed=rows * 3 + cols + d * 5 + bits)
-    x = wl.activations(1, cols, seed=cols + 1, dtype=wl.F16)
+@pytest.mark.parametrize("rows", [8, 148, 301, 1000])
+@pytest.mark.parametrize("cols", [512, 1536, 4608, 17408])
+@pytest.mark.parametrize("batch", [1, 9])
+def test_gemv_tensor_core_path(vqlib, d, bits, rows, cols, batch):
+    """Shapes taken by the tensor-core GEMV (fp16 activations, scale rows of whole 16-byte
+    units): ragged 8-row blocks per CTA, 8 to 272 scale groups per row, tokens in the
+    MMA's first and second row halves, activations from shared and from global memory."""
+    data = wl.uniform_tensor(rows, cols, d, bits, seed=rows * 3 + cols + d * 5 + bits + batch)
+    x = wl.activations(batch, cols, seed=cols + batch, dtype=wl.F16)
     ref = oracle.Tensor(data).linear(x, wl.F16)
     assert_out(run_gemv(vqlib, data, x, wl.F16), ref)
 
 
 @pytest.mark.parametrize("xt", [wl.BF16, wl.F32])
-def test_gemv_row_streaming_other_dtypes(vqlib, xt):
+def test_gemv_non_fp16_activations_large(vqlib, xt):
     data = wl.uniform_tensor(400, 1024, 8, 12, seed=31)
     x = wl.activations(1, 1024, seed=32, dtype=xt)
     ref = oracle.Tensor(data).linear(x, xt)

@@ -11,15 +11,16 @@
 //     expanded weight is used by BT tokens;
 //   * warp 0 (one thread) streams activation tiles [BT][64] into shared memory with TMA
 //     (128-byte swizzle);
-//   * warps 2-5 (128 threads, one weight row each) read the row's packed codes and its
-//     scale for the next 64 columns straight from global memory, look the codes up in
-//     the shared-memory codebook, multiply by the scale (one rounding to the tile type)
-//     and write the 128 x 64 tile in the same 128-byte-swizzled K-major layout, then
-//     fence the generic->async proxy and signal an mbarrier;
+//   * warps 2-9 (256 threads, two per weight row, taking alternate 64-column stages, so
+//     each thread's code prefetch runs two stages ahead) read the row's packed codes and
+//     scale straight from global memory, look the codes up in the shared-memory
+//     codebook, multiply by the scale (one rounding to the tile type) and write the
+//     128 x 64 tile in the same 128-byte-swizzled K-major layout, then fence the
+//     generic->async proxy and signal an mbarrier;
 //   * warp 1 (one thread) issues tcgen05.mma (kind::f16, fp32 accumulation in tensor
 //     memory) for each 64-column stage and frees the stage with tcgen05.commit;
-//   * after the last stage, warps 2-5 read the accumulator out of tensor memory
-//     (tcgen05.ld) and store y.
+//   * after the last stage, warps 2-9 read the accumulator out of tensor memory
+//     (tcgen05.ld; two warps per 32-lane quarter, each half of the columns) and store y.
 // Stages are a ring of STAGES buffers guarded by mbarriers; every wait is bounded and a
 // wait that runs out sets the library's device error word instead of hanging.
 #include <algorithm>
@@ -35,7 +36,7 @@ __device__ unsigned int g_device_error;   // nonzero after a bounded wait ran ou
 
 constexpr int GEMM_BM = 128;       // weight rows per tile (UMMA M)
 constexpr int GEMM_BK = 64;        // columns per stage (one 128-byte swizzle row of 16-bit)
-constexpr int GEMM_THREADS = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 expansion + epilogue
+constexpr int GEMM_THREADS = 320;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 expansion + epilogue
 constexpr int A_TILE_BYTES = GEMM_BM * GEMM_BK * 2;
 
 // Packed codes of one row for one 64-column stage: 64/d codes.
@@ -193,7 +194,9 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
         }
     } else {
         // ---------------- expansion: thread t writes weight row n0 + t of every stage
-        const int t = threadIdx.x - 64;
+        const int et = threadIdx.x - 64;
+        const int t = et & (GEMM_BM - 1);        // tile row
+        const int par = et >> 7;                 // this thread expands stages kb = par, par + 2, ...
         const int row = n0 + t;
         const bool rv = row < W.rows;
         const uint8_t *crow = codes_e + (int64_t)(rv ? row : 0) * W.code_row_bytes;
@@ -203,10 +206,10 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
 
         Blk cur, nxt;
         __half sc_cur = __float2half(0.f), sc_nxt = __float2half(0.f);
-        if (rv) { cur.load(crow, 0); sc_cur = srow[0]; } else cur.zero();
-        for (int kb = 0; kb < nkb; kb++) {
-            if (kb + 1 < nkb) {
-                if (rv) { nxt.load(crow, kb + 1); sc_nxt = srow[kb + 1]; } else nxt.zero();
+        if (rv && par < nkb) { cur.load(crow, par); sc_cur = srow[par]; } else cur.zero();
+        for (int kb = par; kb < nkb; kb += 2) {
+            if (kb + 2 < nkb) {
+                if (rv) { nxt.load(crow, kb + 2); sc_nxt = srow[kb + 2]; } else nxt.zero();
             }
             const int s = kb % STAGES, r = kb / STAGES;
             const bool ok = r == 0 || mbar_wait(&empty[s], (r - 1) & 1);
@@ -258,8 +261,10 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
         if (__all_sync(0xffffffffu, waited && !*abort_flag)) {   // warp-uniform: tcgen05.ld is .sync.aligned
             const int q = warp & 3;                  // TMEM lanes 32q..32q+31 belong to this warp
             const int erow = n0 + q * 32 + lane;
+            const int chalf = (warp - 2) >> 2;       // two warps per quarter: each takes half the columns
+            constexpr int CW = BT / 2 >= 32 ? BT / 2 : 32;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BT; c0 += 32) {
+            for (int c0 = chalf * CW; c0 < BT && c0 < (chalf + 1) * CW; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
                 tmem_ld_wait();

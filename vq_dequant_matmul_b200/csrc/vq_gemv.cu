@@ -288,13 +288,13 @@ static vq_status run_x(const Mat &W, const void *x, int batch, void *y, int yt, 
     }
 }
 
-vq_status launch_gemv_stream(const Mat &W, const void *x, vq_dtype xt, void *y, vq_dtype yt, cudaStream_t s);
+vq_status launch_gemv_mma(const Mat &W, const void *x, vq_dtype xt, int batch, void *y, vq_dtype yt, cudaStream_t s);
 
 vq_status launch_gemv(const Mat &W, const void *x, vq_dtype xt, int batch, void *y, vq_dtype yt,
                       cudaStream_t s)
 {
-    if (batch == 1) {
-        const vq_status st = launch_gemv_stream(W, x, xt, y, yt, s);
+    {   // tensor-core path for fp16 activations
+        const vq_status st = launch_gemv_mma(W, x, xt, batch, y, yt, s);
         if (st != VQ_ERR_UNSUPPORTED) return st;
     }
     if (xt == VQ_F16) return run_x<__half>(W, x, batch, y, (int)yt, s);
