@@ -210,7 +210,7 @@ def run_ours(args, rank, world, local_rank):
     prefill_tflops = sum(pre_flops) * world / (pre_ms * 1e-3) / 1e12
 
     gemv_gbs = sum(dec_bytes) / (sum(kern_ms[:3]) * 1e-3) / 1e9
-    roofline = {"kernel": "gemv_stream_kernel<2,8,half>", "bound": "hbm", "achieved": round(gemv_gbs, 1),
+    roofline = {"kernel": "gemv_mma_kernel<2,8> (mma.sync GEMV)", "bound": "hbm", "achieved": round(gemv_gbs, 1),
                 "peak": pk["hbm"], "unit": "GB/s", "frac": round(gemv_gbs / pk["hbm"], 4),
                 "traffic": args.traffic, "peak_source": pk["source"] + " (burst copy)",
                 "per_projection_gbs": [round(dec_bytes[i] / (kern_ms[i] * 1e-3) / 1e9, 1) for i in range(3)],

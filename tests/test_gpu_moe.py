@@ -116,3 +116,38 @@ def test_c5_moe_layer(vqlib, T):
     toks = np.arange(T) if T <= 8 else np.random.default_rng(T).choice(T, 8, replace=False)
     ref, _ = oracle_moe(mw, x, wl.F16, ids, w, toks)
     assert normwise(to_np(y)[toks], ref) <= NORMWISE_TOL
+
+
+def test_moe_decode_path_token_chunks(vqlib):
+    """Few tokens per expert on average (the tensor-core GEMV route) but one expert holds
+    40 tokens: its tokens go through the MMA rows in chunks of 16."""
+    mw = small_moe(E=64, seed=14, topk=1, hidden=512, inter=512)
+    x, _, _ = wl.moe_inputs(mw, 40, seed=15)
+    ids = np.full((40, 1), 3, np.int32)
+    ids[::7, 0] = 5
+    w = np.ones((40, 1), np.float32)
+    y, st = run_moe(vqlib, mw, x, wl.F16, ids, w)
+    ref, _ = oracle_moe(mw, x, wl.F16, ids, w, np.arange(40))
+    assert st == 0 and normwise(to_np(y), ref) <= NORMWISE_TOL
+
+
+@pytest.mark.parametrize("T", [1, 2, 7])
+def test_moe_decode_path_bf16(vqlib, T):
+    mw = small_moe(seed=16 + T, topk=2, E=16, hidden=512, inter=512)
+    x, ids, w = wl.moe_inputs(mw, T, seed=17, dtype=wl.BF16)
+    y, st = run_moe(vqlib, mw, x, wl.BF16, ids, w)
+    ref, _ = oracle_moe(mw, x, wl.BF16, ids, w, np.arange(T))
+    assert st == 0 and normwise(to_np(y), ref) <= NORMWISE_TOL
+
+
+@pytest.mark.parametrize("T", [1, 3, 6])
+@pytest.mark.parametrize("geoms", [((8, 12), (4, 8), (4, 12)), ((2, 8), (2, 8), (2, 8)), ((4, 12), (8, 8), (2, 12))])
+def test_moe_decode_path_geometries(vqlib, T, geoms):
+    """Layers whose scale rows are whole 16-byte units, few tokens per expert: the grouped
+    tensor-core GEMV route, mixed tiers in one launch."""
+    mw = small_moe(geoms=geoms, seed=20 + T, E=16, hidden=1024, inter=512)
+    x, ids, w = wl.moe_inputs(mw, T, seed=T + 200)
+    y, st = run_moe(vqlib, mw, x, wl.F16, ids, w)
+    ref, bad = oracle_moe(mw, x, wl.F16, ids, w, np.arange(T))
+    assert st == 0 and bad == 0
+    assert normwise(to_np(y), ref) <= NORMWISE_TOL

@@ -23,16 +23,48 @@ struct SmemCB {
     static constexpr int BYTES = K * STRIDE;
 
     // Copy the global [K][D] fp16 table into shared memory, NREP copies interleaved:
-    // word index ((e * NREP + rep) * D/2 + part) holds word `part` of entry e.
-    __device__ static void stage(uint8_t *smem, const __half *gcb) {
-        constexpr int WPE = D / 2;
-        constexpr int TOTAL = K * NREP * WPE;
-        const uint32_t *g = reinterpret_cast<const uint32_t *>(gcb);
-        uint32_t *s = reinterpret_cast<uint32_t *>(smem);
-        for (int w = threadIdx.x; w < TOTAL; w += blockDim.x) {
-            int e = w / (NREP * WPE);
-            int part = w % WPE;
-            s[w] = __ldg(g + e * WPE + part);
+    // entry e occupies bytes [e * STRIDE, (e + 1) * STRIDE), copy `rep` at rep * ENTRY.
+    // Every global load is issued before the shared stores that use it, so a CTA pays
+    // about one memory latency per pass instead of one per word.
+    __device__ static void stage(uint8_t *smem, const __half *gcb) { stage(smem, gcb, threadIdx.x, blockDim.x); }
+
+    // The same with an explicit thread index / count (a subset of the block stages it).
+    __device__ static void stage(uint8_t *smem, const __half *gcb, int tid, int nthreads) {
+        if constexpr (NREP > 1) {
+            static_assert(STRIDE == 128, "replicated entries span 128 bytes");
+            for (int e = tid; e < K; e += nthreads) {
+                uint4 v;
+                if constexpr (D == 2) {
+                    const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(gcb) + e);
+                    v = make_uint4(w, w, w, w);
+                } else if constexpr (D == 4) {
+                    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(gcb) + e);
+                    v = make_uint4(w.x, w.y, w.x, w.y);
+                } else {
+                    v = __ldg(reinterpret_cast<const uint4 *>(gcb) + e);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(smem + (size_t)e * STRIDE);
+#pragma unroll
+                for (int i = 0; i < 8; i++) dst[i] = v;
+            }
+        } else {
+            constexpr int N16 = K * D * 2 / 16;
+            const uint4 *g = reinterpret_cast<const uint4 *>(gcb);
+            uint4 *dst = reinterpret_cast<uint4 *>(smem);
+            constexpr int B = 8;   // loads in flight per thread
+            for (int i0 = tid; i0 < N16; i0 += B * nthreads) {
+                uint4 v[B];
+#pragma unroll
+                for (int j = 0; j < B; j++) {
+                    const int i = i0 + j * nthreads;
+                    if (i < N16) v[j] = __ldg(g + i);
+                }
+#pragma unroll
+                for (int j = 0; j < B; j++) {
+                    const int i = i0 + j * nthreads;
+                    if (i < N16) dst[i] = v[j];
+                }
+            }
         }
     }
 };

@@ -28,14 +28,11 @@
 // across warps in a fixed order (deterministic).
 #include <algorithm>
 
-#include "vq_codebook.cuh"
-#include "vq_internal.cuh"
-#include "vq_sm100.cuh"
+#include "vq_mma.cuh"
 
 namespace vq {
 
 constexpr int MMAV_MAX_THREADS = 32 * 17;   // producer warp + up to 16 consumer warps
-constexpr int MMAV_ROWS = 8;                // rows per block (the MMA's n)
 
 struct MmaGemvCfg {
     int NW;              // consumer warps
@@ -45,92 +42,6 @@ struct MmaGemvCfg {
     int stage_bytes;     // bytes of one stage (8 row slots + 8 rows of scales)
     int x_bytes;         // activations in shared memory (cols * 2, rounded to 16)
     unsigned int *err;
-};
-
-__device__ __forceinline__ void mma_f16_f32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint32_t lds16(uint32_t a) {
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
-    return v;
-}
-
-__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void bar_sync_named(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// The lane's codes of one scale group (64 columns) of its row, as they are needed by
-// the four MMAs: code(j) for j < 64 / d / 4.
-template <int D, int BITS>
-struct LaneCodes {
-    uint32_t w0, w1, w2;
-    int sh;   // 12-bit d = 4 / d = 8: bit offset inside w0:w1
-    __device__ __forceinline__ void load(uint32_t grp_addr, int t) {
-        if constexpr (BITS == 8) {
-            if constexpr (D == 2) { const uint2 v = lds64(grp_addr + 8 * t); w0 = v.x; w1 = v.y; }
-            else if constexpr (D == 4) { w0 = lds32(grp_addr + 4 * t); }
-            else { w0 = lds16(grp_addr + 2 * t); }
-        } else {
-            if constexpr (D == 2) {          // 12 bytes at 12t: codes at bits 12j
-                w0 = lds32(grp_addr + 12 * t);
-                w1 = lds32(grp_addr + 12 * t + 4);
-                w2 = lds32(grp_addr + 12 * t + 8);
-            } else if constexpr (D == 4) {   // 48 bits at bit 48t
-                const int wi = (3 * t) >> 1;
-                sh = 16 * (t & 1);
-                w0 = lds32(grp_addr + 4 * wi);
-                w1 = lds32(grp_addr + 4 * wi + 4);
-            } else {                         // 24 bits at bit 24t
-                const int bit = 24 * t;
-                sh = bit & 31;
-                w0 = lds32(grp_addr + 4 * (bit >> 5));
-                w1 = lds32(grp_addr + 4 * (bit >> 5) + 4);
-            }
-        }
-    }
-    __device__ __forceinline__ uint32_t code(int j) const {
-        if constexpr (BITS == 8) {
-            if constexpr (D == 2) return ((j < 4 ? w0 : w1) >> (8 * (j & 3))) & 0xFFu;
-            else return (w0 >> (8 * j)) & 0xFFu;
-        } else {
-            if constexpr (D == 2) {
-                const int bit = 12 * j, wi = bit >> 5, s = bit & 31;
-                const uint32_t lo = wi == 0 ? w0 : wi == 1 ? w1 : w2;
-                const uint32_t hi = wi == 0 ? w1 : w2;
-                return (s + 12 <= 32 ? (lo >> s) : __funnelshift_r(lo, hi, s)) & 0xFFFu;
-            } else {
-                const uint64_t v = ((uint64_t)w1 << 32) | w0;
-                return (uint32_t)(v >> (sh + 12 * j)) & 0xFFFu;
-            }
-        }
-    }
 };
 
 // NT = 1: tokens 0..7 (the MMA's rows g); NT = 2: tokens 0..15 (rows g and g + 8).
@@ -147,9 +58,12 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
     uint8_t *sX = sCB + CB::BYTES;
     uint8_t *sStage = sX + cfg.x_bytes;
     constexpr int NTOK = 8 * NT;
-    float *red = reinterpret_cast<float *>(sStage + (size_t)cfg.STAGES * cfg.stage_bytes);   // [2][NW][NTOK][8]
-    uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * cfg.NW * NTOK * MMAV_ROWS);
+    // partial sums: a ring of STAGES + 1 buffers [NW][NTOK][8] (a consumer warp is at most
+    // STAGES - 1 blocks ahead of the slowest one, so a buffer is never rewritten while read)
+    float *red = reinterpret_cast<float *>(sStage + (size_t)cfg.STAGES * cfg.stage_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(red + (cfg.STAGES + 1) * cfg.NW * NTOK * MMAV_ROWS);
     uint64_t *empty = full + cfg.STAGES;
+    uint64_t *red_bar = empty + cfg.STAGES;   // [STAGES + 1]: partials of a block posted (one arrive per warp)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nblk_total = (W.rows + MMAV_ROWS - 1) / MMAV_ROWS;
@@ -169,6 +83,7 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], cfg.NW);
         }
+        for (int s = 0; s <= cfg.STAGES; s++) mbar_init(&red_bar[s], cfg.NW);
         mbar_fence_init();
     }
     __syncthreads();
@@ -220,47 +135,25 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
         const uint32_t stage = smem_u32(sStage + (size_t)slot * cfg.stage_bytes);
         const uint32_t row_lane = stage + g * cfg.slot_stride;
         const uint32_t sc_base = stage + MMAV_ROWS * cfg.slot_stride;
+        const uint32_t sc0 = sc_base + (2 * t) * (int)W.scale_row_elems * 2;   // scales of rows 2t, 2t + 1
+        const uint32_t sc1 = sc0 + (int)W.scale_row_elems * 2;
         float tot[2][2] = {{0.f, 0.f}, {0.f, 0.f}};   // [token g / g + 8][row 2t / 2t + 1]
         if (!dead) {
             for (int grp = cw; grp < G; grp += cfg.NW) {
-                LaneCodes<D, BITS> lc;
-                lc.load(row_lane + grp * GB, t);
                 uint32_t x0[8], x1[8];
-                {
-                    uint4 p, q;
-                    if constexpr (XS) { p = lds128(xs0 + grp * 128); q = lds128(xs0 + grp * 128 + 16); }
-                    else { p = __ldg(reinterpret_cast<const uint4 *>(xg0 + grp * 64)); q = __ldg(reinterpret_cast<const uint4 *>(xg0 + grp * 64) + 1); }
-                    x0[0] = p.x; x0[1] = p.y; x0[2] = p.z; x0[3] = p.w; x0[4] = q.x; x0[5] = q.y; x0[6] = q.z; x0[7] = q.w;
-                }
+                if constexpr (XS) lds_x16(xs0 + grp * 128, x0);
+                else ldg_x16(xg0 + grp * 64, x0);
                 if constexpr (NT == 2) {
-                    uint4 p, q;
-                    if constexpr (XS) { p = lds128(xs1 + grp * 128); q = lds128(xs1 + grp * 128 + 16); }
-                    else { p = __ldg(reinterpret_cast<const uint4 *>(xg1 + grp * 64)); q = __ldg(reinterpret_cast<const uint4 *>(xg1 + grp * 64) + 1); }
-                    x1[0] = p.x; x1[1] = p.y; x1[2] = p.z; x1[3] = p.w; x1[4] = q.x; x1[5] = q.y; x1[6] = q.z; x1[7] = q.w;
+                    if constexpr (XS) lds_x16(xs1 + grp * 128, x1);
+                    else ldg_x16(xg1 + grp * 64, x1);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 8; i++) x1[i] = x0[i];
                 }
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int s = 0; s < 4; s++) {
-                    const uint32_t a[4] = {x0[2 * s], x1[2 * s], x0[2 * s + 1], x1[2 * s + 1]};
-                    uint32_t b0, b1;
-                    if constexpr (D == 2) {
-                        b0 = lds32(cb_lane + lc.code(2 * s) * CB::STRIDE);
-                        b1 = lds32(cb_lane + lc.code(2 * s + 1) * CB::STRIDE);
-                    } else if constexpr (D == 4) {
-                        const uint2 e = lds64(cb_lane + lc.code(s) * CB::STRIDE);
-                        b0 = e.x; b1 = e.y;
-                    } else {
-                        const uint4 e = lds128(cb_lane + lc.code(s >> 1) * CB::STRIDE);
-                        b0 = (s & 1) ? e.z : e.x;
-                        b1 = (s & 1) ? e.w : e.y;
-                    }
-                    mma_f16_f32(d, a, b0, b1);
-                }
-                const float s0 = __half2float(__ushort_as_half((unsigned short)lds16(sc_base + ((2 * t) * (int)W.scale_row_elems + grp) * 2)));
-                const float s1 = __half2float(__ushort_as_half((unsigned short)lds16(sc_base + ((2 * t + 1) * (int)W.scale_row_elems + grp) * 2)));
+                float d[4];
+                mma_group<D, BITS>(row_lane + grp * GB, t, cb_lane, x0, x1, d);
+                const float s0 = __half2float(__ushort_as_half((unsigned short)lds16(sc0 + grp * 2)));
+                const float s1 = __half2float(__ushort_as_half((unsigned short)lds16(sc1 + grp * 2)));
                 tot[0][0] = fmaf(s0, d[0], tot[0][0]);
                 tot[0][1] = fmaf(s1, d[1], tot[0][1]);
                 if constexpr (NT == 2) {
@@ -271,21 +164,33 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
-        // red[buf][cw][token][row]
-        float *rb = red + (k & 1) * cfg.NW * NTOK * MMAV_ROWS;
+        // post partials [cw][token][row] (phase-tracked: one mbarrier per ring buffer);
+        // warp 0 alone waits for all warps' partials of the block and reduces them
+        const int rbi = k % (cfg.STAGES + 1);
+        float *rb = red + rbi * cfg.NW * NTOK * MMAV_ROWS;
         rb[(cw * NTOK + g) * MMAV_ROWS + 2 * t] = tot[0][0];
         rb[(cw * NTOK + g) * MMAV_ROWS + 2 * t + 1] = tot[0][1];
         if constexpr (NT == 2) {
             rb[(cw * NTOK + g + 8) * MMAV_ROWS + 2 * t] = tot[1][0];
             rb[(cw * NTOK + g + 8) * MMAV_ROWS + 2 * t + 1] = tot[1][1];
         }
-        bar_sync_named(1, cfg.NW * 32);
-        for (int q = cw * 32 + lane; q < NTOK * MMAV_ROWS; q += cfg.NW * 32) {   // (token, row) outputs
-            const int tok = q / MMAV_ROWS, rr = q % MMAV_ROWS;
-            float v = 0.f;
-            for (int w = 0; w < cfg.NW; w++) v += rb[(w * NTOK + tok) * MMAV_ROWS + rr];
-            const int r = (b_begin + k) * MMAV_ROWS + rr;
-            if (r < W.rows && tok < batch) store_out(y, (int64_t)tok * W.rows + r, v, yt);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_bar[rbi]);
+        if (cw == 0) {
+            const bool ok = mbar_wait(&red_bar[rbi], (k / (cfg.STAGES + 1)) & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicExch(cfg.err, 1u);
+                dead = true;
+            }
+            if (!dead) {
+                for (int q = lane; q < NTOK * MMAV_ROWS; q += 32) {   // (token, row) outputs
+                    const int tok = q / MMAV_ROWS, rr = q % MMAV_ROWS;
+                    float v = 0.f;
+                    for (int w = 0; w < cfg.NW; w++) v += rb[(w * NTOK + tok) * MMAV_ROWS + rr];
+                    const int r = (b_begin + k) * MMAV_ROWS + rr;
+                    if (r < W.rows && tok < batch) store_out(y, (int64_t)tok * W.rows + r, v, yt);
+                }
+            }
         }
     }
     (void)scale_bytes;
@@ -355,11 +260,12 @@ vq_status launch_gemv_mma(const Mat &W, const void *x, vq_dtype xt, int batch, v
     c.x_bytes = xb <= 49152 ? (int)((xb + 15) / 16 * 16) : 0;
     const size_t cb = mmav_cb_bytes(W.d, W.bits);
     const int ntok = batch <= 8 ? 8 : 16;
-    const size_t fixed = 128 + cb + c.x_bytes + 2 * (size_t)c.NW * ntok * MMAV_ROWS * 4;
+    const size_t fixed = 128 + cb + c.x_bytes + (size_t)c.NW * ntok * MMAV_ROWS * 4 + 8;   // + one red buffer
+    const size_t per_stage = (size_t)c.stage_bytes + (size_t)c.NW * ntok * MMAV_ROWS * 4 + 3 * 8;
     c.STAGES = 8;
-    while (c.STAGES >= 2 && fixed + (size_t)c.STAGES * (c.stage_bytes + 16) > 232448) c.STAGES--;
+    while (c.STAGES >= 2 && fixed + (size_t)c.STAGES * per_stage > 232448) c.STAGES--;
     if (c.STAGES < 2) return VQ_ERR_UNSUPPORTED;
-    const size_t smem = fixed + (size_t)c.STAGES * (c.stage_bytes + 16);
+    const size_t smem = fixed + (size_t)c.STAGES * per_stage;
     c.err = device_error_word();
     if (!c.err) return VQ_ERR_CUDA;
     const int nblk = (W.rows + MMAV_ROWS - 1) / MMAV_ROWS;

@@ -11,8 +11,10 @@
 //      exclusive scan, stable scatter of pair indices ordered by (expert, token, slot),
 //      the list of active experts and a tile list (expert, first row, rows);
 //   2. gate/up: ONE grouped launch over (projection, active expert, row block) — each
-//      projection with its own geometry, so mixed tiers share the launch;
-//   3. down: one grouped launch with input silu(g) * u formed on the fly;
+//      projection with its own geometry, so mixed tiers share the launch.  Few tokens
+//      per expert (decode): the tensor-core GEMV with the expert's tokens as MMA rows;
+//      several per expert (prefill): the tcgen05 GEMM over a tile list;
+//   3. h = silu(g) * u in fp16, then down: one grouped launch of the same kind;
 //   4. combine: y_t = sum over slots (in order) of w * o, skipping invalid pairs.
 // Pairs whose expert id is outside [0, E) are counted in the workspace status word and
 // contribute nothing.  Float atomics are never used: results are deterministic.
@@ -21,7 +23,7 @@
 
 #include "vq_codebook.cuh"
 #include "vq_gemm_api.cuh"
-#include "vq_gemv_body.cuh"
+#include "vq_mma.cuh"
 #include "vq_internal.cuh"
 
 namespace vq {
@@ -185,79 +187,205 @@ __global__ void __launch_bounds__(BUCKET_THREADS) moe_bucket_kernel(BucketArgs a
     }
 }
 
-// ------------------------------------------------------------------ 2./3. grouped GEMV
+// ------------------------------------------------------------------ 2./3. grouped tensor-core GEMV (decode)
 
-struct MoeGemvArgs {
-    Mat W[2];
-    float *out[2];                    // [P][W.rows] fp32, rows in bucket order
-    const void *x;                    // stage 1: activations [T][hidden]
-    const float *g, *u;               // stage 2: [P][inter]
+// Grouped decode projections on the tensor-core GEMV: persistent CTAs take balanced,
+// contiguous ranges of items (projection p, active expert, 8-row block) in that order;
+// an item's rows arrive by bulk copy in a ring of stages; consumer warps split the
+// block's 64-column groups, with the expert's tokens (up to 16 at a time) as the MMA's A
+// rows.  The codebook is restaged only when the projection (or, for per-expert
+// codebooks, the expert) changes.
+constexpr int MOE_MMA_MAX_THREADS = 32 * 9;   // producer warp + 8 consumer warps
+
+struct MoeMmaArgs {
+    Mat W[3];
+    int nproj;
+    float *out[3];               // [P][W[p].rows], rows in bucket order
+    const __half *ain[3];        // A rows: x by token (stage 1) or h by bucket position
+    int a_by_token[3];
     const int *sorted, *offsets, *act, *nact;
     int topk;
+    int NW, STAGES, slot_stride, stage_bytes;
+    unsigned int *err;
 };
 
-template <int D, int BITS, int XMODE>
-__device__ __forceinline__ void moe_gemv_body(const MoeGemvArgs &a, const Mat &W, int e, float *out, uint8_t *smem)
-{
-    using CB = SmemCB<D, BITS>;
-    using S = B1Shape<D, BITS>;
-    constexpr int R = S::R;
-    const int nchunk = (W.cols / D + S::CPC - 1) / S::CPC;
-    int lpr_log2 = 0;
-    while ((1 << lpr_log2) < 32 && (1 << lpr_log2) < nchunk) lpr_log2++;
-    const int LPR = 1 << lpr_log2, G = 32 >> lpr_log2;
-    const int rows_per_cta = GEMV_BODY_WARPS * R * G;
-    const int row0 = blockIdx.x * rows_per_cta;
-    if (row0 >= W.rows) return;                          // uniform over the block
+struct MoeItem {
+    int p, e, blk;
+};
 
-    CB::stage(smem, W.codebook + (int64_t)e * W.expert_codebook_stride);
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> lpr_log2, l = lane & (LPR - 1);
-    const int rbase = row0 + warp * R * G + g * R;
-    const uint8_t *codes = W.codes + (int64_t)e * W.expert_code_stride;
-    const __half *scales = W.scales + (int64_t)e * W.expert_scale_stride;
-    const uint8_t *cbase = smem + (lane % CB::NREP) * CB::ENTRY;
-    const int j_end = a.offsets[e + 1];
-    for (int j = a.offsets[e]; j < j_end; j++) {
-        float acc[R];
-#pragma unroll
-        for (int i = 0; i < R; i++) acc[i] = 0.f;
-        if constexpr (XMODE == 2) {
-            const int inter = W.cols;
-            b1_accumulate<D, BITS>(codes, scales, W.rows, W.cols, W.code_row_bytes, W.scale_row_elems, cbase,
-                                   rbase, l, LPR, XSiluMul{a.g + (int64_t)j * inter, a.u + (int64_t)j * inter},
-                                   acc);
-        } else {
-            using XT = typename std::conditional<XMODE == 0, __half, __nv_bfloat16>::type;
-            const int t = a.sorted[j] / a.topk;
-            b1_accumulate<D, BITS>(codes, scales, W.rows, W.cols, W.code_row_bytes, W.scale_row_elems, cbase,
-                                   rbase, l, LPR, XRow<XT>{(const XT *)a.x + (int64_t)t * W.cols}, acc);
+__device__ __forceinline__ MoeItem moe_item(const MoeMmaArgs &a, int i, int nact) {
+    MoeItem it{0, 0, 0};
+    for (int p = 0; p < a.nproj; p++) {
+        const int nb = (a.W[p].rows + MMAV_ROWS - 1) / MMAV_ROWS;
+        if (i < nact * nb) {
+            it.p = p;
+            it.e = a.act[i / nb];
+            it.blk = i % nb;
+            return it;
         }
-#pragma unroll
-        for (int i = 0; i < R; i++) {
-            const float v = group_sum(acc[i], LPR);
-            if (l == 0 && rbase + i < W.rows) out[(int64_t)j * W.rows + rbase + i] = v;
-        }
+        i -= nact * nb;
+    }
+    return it;
+}
+
+template <int D, int BITS>
+__device__ __forceinline__ void moe_mma_chunk(const MoeMmaArgs &a, const Mat &W, int p, uint32_t stage,
+                                              uint32_t cb_lane, int cw, int lane, int c0, int j1, float (&tot)[2][2])
+{
+    constexpr int GB = (64 / D) * BITS / 8;
+    const int g = lane >> 2, t = lane & 3;
+    const int G = W.cols / 64;
+    const int pos0 = min(c0 + g, j1 - 1), pos1 = min(c0 + g + 8, j1 - 1);
+    const __half *r0, *r1;
+    if (a.a_by_token[p]) {
+        r0 = a.ain[p] + (int64_t)(a.sorted[pos0] / a.topk) * W.cols;
+        r1 = a.ain[p] + (int64_t)(a.sorted[pos1] / a.topk) * W.cols;
+    } else {
+        r0 = a.ain[p] + (int64_t)pos0 * W.cols;
+        r1 = a.ain[p] + (int64_t)pos1 * W.cols;
+    }
+    r0 += 16 * t;
+    r1 += 16 * t;
+    const uint32_t row_lane = stage + g * a.slot_stride;
+    const uint32_t sc_base = stage + MMAV_ROWS * a.slot_stride;
+    for (int grp = cw; grp < G; grp += a.NW) {
+        uint32_t x0[8], x1[8];
+        ldg_x16(r0 + grp * 64, x0);
+        ldg_x16(r1 + grp * 64, x1);
+        float d[4];
+        mma_group<D, BITS>(row_lane + grp * GB, t, cb_lane, x0, x1, d);
+        const float s0 = __half2float(__ushort_as_half((unsigned short)lds16(sc_base + ((2 * t) * (int)W.scale_row_elems + grp) * 2)));
+        const float s1 = __half2float(__ushort_as_half((unsigned short)lds16(sc_base + ((2 * t + 1) * (int)W.scale_row_elems + grp) * 2)));
+        tot[0][0] = fmaf(s0, d[0], tot[0][0]);
+        tot[0][1] = fmaf(s1, d[1], tot[0][1]);
+        tot[1][0] = fmaf(s0, d[2], tot[1][0]);
+        tot[1][1] = fmaf(s1, d[3], tot[1][1]);
     }
 }
 
-template <int XMODE>
-__global__ void __launch_bounds__(GEMV_BODY_THREADS) moe_gemv_kernel(MoeGemvArgs a)
+__global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaArgs a)
 {
-    extern __shared__ __align__(16) uint8_t smem[];
-    if ((int)blockIdx.y >= *a.nact) return;
-    const int e = a.act[blockIdx.y];
-    const Mat &W = a.W[blockIdx.z];
-    float *out = a.out[blockIdx.z];
-    switch (geom_of(W.d, W.bits)) {
-    case G_D2_B8: moe_gemv_body<2, 8, XMODE>(a, W, e, out, smem); break;
-    case G_D4_B8: moe_gemv_body<4, 8, XMODE>(a, W, e, out, smem); break;
-    case G_D8_B8: moe_gemv_body<8, 8, XMODE>(a, W, e, out, smem); break;
-    case G_D2_B12: moe_gemv_body<2, 12, XMODE>(a, W, e, out, smem); break;
-    case G_D4_B12: moe_gemv_body<4, 12, XMODE>(a, W, e, out, smem); break;
-    case G_D8_B12: moe_gemv_body<8, 12, XMODE>(a, W, e, out, smem); break;
-    default: break;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *sCB = smem;
+    uint8_t *sStage = sCB + SmemCB<8, 12>::BYTES;            // largest table (64 KB)
+    float *red = reinterpret_cast<float *>(sStage + (size_t)a.STAGES * a.stage_bytes);   // [2][NW][16][8]
+    uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * a.NW * 16 * MMAV_ROWS);
+    uint64_t *empty = full + a.STAGES;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nact = *a.nact;
+    int N = 0;
+    for (int p = 0; p < a.nproj; p++) N += nact * ((a.W[p].rows + MMAV_ROWS - 1) / MMAV_ROWS);
+    const int i_begin = (int)(((int64_t)N * blockIdx.x) / gridDim.x);
+    const int i_end = (int)(((int64_t)N * (blockIdx.x + 1)) / gridDim.x);
+    if (i_begin >= i_end) return;                               // uniform over the CTA
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < a.STAGES; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], a.NW);
+        }
+        mbar_fence_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int i = i_begin, k = 0; i < i_end; i++, k++) {
+                const int slot = k % a.STAGES, round = k / a.STAGES;
+                if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1)) {
+                    atomicExch(a.err, 1u);
+                    break;
+                }
+                const MoeItem it = moe_item(a, i, nact);
+                const Mat &W = a.W[it.p];
+                const int r0 = it.blk * MMAV_ROWS;
+                const int nrows = min(MMAV_ROWS, W.rows - r0);
+                const uint8_t *codes = W.codes + (int64_t)it.e * W.expert_code_stride;
+                const __half *scales = W.scales + (int64_t)it.e * W.expert_scale_stride;
+                const uint32_t base = smem_u32(sStage + (size_t)slot * a.stage_bytes);
+                mbar_arrive_expect_tx(&full[slot], (uint32_t)(nrows * (W.code_row_bytes + W.scale_row_elems * 2)));
+                for (int r = 0; r < nrows; r++)
+                    bulk_copy_g2s(base + r * a.slot_stride, codes + (int64_t)(r0 + r) * W.code_row_bytes,
+                                  (uint32_t)W.code_row_bytes, &full[slot]);
+                bulk_copy_g2s(base + MMAV_ROWS * a.slot_stride, scales + (int64_t)r0 * W.scale_row_elems,
+                              (uint32_t)(nrows * W.scale_row_elems * 2), &full[slot]);
+            }
+        }
+        return;
+    }
+
+    const int cw = warp - 1;
+    const int nthr = a.NW * 32;
+    const __half *cur_cb = nullptr;
+    bool dead = false;
+    int rbuf = 0;
+    for (int i = i_begin, k = 0; i < i_end; i++, k++) {
+        const int slot = k % a.STAGES, round = k / a.STAGES;
+        const MoeItem it = moe_item(a, i, nact);
+        const Mat &W = a.W[it.p];
+        const int geom = geom_of(W.d, W.bits);
+        const __half *cb = W.codebook + (int64_t)it.e * W.expert_codebook_stride;
+        if (cb != cur_cb) {                                     // (re)stage the codebook
+            bar_sync_named(1, nthr);
+            switch (geom) {
+            case G_D2_B8: SmemCB<2, 8>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
+            case G_D4_B8: SmemCB<4, 8>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
+            case G_D8_B8: SmemCB<8, 8>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
+            case G_D2_B12: SmemCB<2, 12>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
+            case G_D4_B12: SmemCB<4, 12>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
+            default: SmemCB<8, 12>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
+            }
+            bar_sync_named(1, nthr);
+            cur_cb = cb;
+        }
+        if (!dead) {
+            const bool ok = mbar_wait(&full[slot], round & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicExch(a.err, 1u);
+                dead = true;
+            }
+        }
+        const uint32_t stage = smem_u32(sStage + (size_t)slot * a.stage_bytes);
+        const int j0 = a.offsets[it.e], j1 = a.offsets[it.e + 1];
+        const int r0 = it.blk * MMAV_ROWS;
+        for (int c0 = j0; c0 < j1; c0 += 16) {
+            float tot[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            if (!dead) {
+                switch (geom) {
+#define VQ_MOE_CASE(GG, DD, BB)                                                                              \
+    case GG: moe_mma_chunk<DD, BB>(a, W, it.p, stage, smem_u32(sCB) + (lane % SmemCB<DD, BB>::NREP) *       \
+                                   SmemCB<DD, BB>::ENTRY, cw, lane, c0, j1, tot); break;
+                VQ_MOE_CASE(G_D2_B8, 2, 8)
+                VQ_MOE_CASE(G_D4_B8, 4, 8)
+                VQ_MOE_CASE(G_D8_B8, 8, 8)
+                VQ_MOE_CASE(G_D2_B12, 2, 12)
+                VQ_MOE_CASE(G_D4_B12, 4, 12)
+                VQ_MOE_CASE(G_D8_B12, 8, 12)
+#undef VQ_MOE_CASE
+                default: break;
+                }
+            }
+            if (c0 + 16 >= j1) {                                // last read of this stage
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
+            }
+            float *rb = red + rbuf * a.NW * 16 * MMAV_ROWS;
+            const int g = lane >> 2, t = lane & 3;
+            rb[(cw * 16 + g) * MMAV_ROWS + 2 * t] = tot[0][0];
+            rb[(cw * 16 + g) * MMAV_ROWS + 2 * t + 1] = tot[0][1];
+            rb[(cw * 16 + g + 8) * MMAV_ROWS + 2 * t] = tot[1][0];
+            rb[(cw * 16 + g + 8) * MMAV_ROWS + 2 * t + 1] = tot[1][1];
+            bar_sync_named(1, nthr);
+            for (int q = cw * 32 + lane; q < 16 * MMAV_ROWS; q += nthr) {
+                const int tk = q / MMAV_ROWS, rr = q % MMAV_ROWS;
+                float v = 0.f;
+                for (int w = 0; w < a.NW; w++) v += rb[(w * 16 + tk) * MMAV_ROWS + rr];
+                if (c0 + tk < j1 && r0 + rr < W.rows) a.out[it.p][(int64_t)(c0 + tk) * W.rows + r0 + rr] = v;
+            }
+            rbuf ^= 1;
+        }
     }
 }
 
@@ -332,41 +460,37 @@ __global__ void moe_combine_kernel(const float *__restrict__ o, const int *__res
 // ------------------------------------------------------------------ host
 
 
-static size_t cb_smem_bytes(const Mat &W) {
-    switch (geom_of(W.d, W.bits)) {
-    case G_D2_B8: return SmemCB<2, 8>::BYTES;
-    case G_D4_B8: return SmemCB<4, 8>::BYTES;
-    case G_D8_B8: return SmemCB<8, 8>::BYTES;
-    case G_D2_B12: return SmemCB<2, 12>::BYTES;
-    case G_D4_B12: return SmemCB<4, 12>::BYTES;
-    default: return SmemCB<8, 12>::BYTES;
-    }
+unsigned int *device_error_word();
+
+static int moe_num_sms() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
 }
 
-static int gemv_rows_per_cta(const Mat &W) {
-    const int bits = W.bits, d = W.d;
-    const int cpc = bits == 8 ? 16 : 32, R = bits == 8 ? 8 : 4;
-    const int nchunk = (W.cols / d + cpc - 1) / cpc;
-    int lpr = 1;
-    while (lpr < 32 && lpr < nchunk) lpr *= 2;
-    return GEMV_BODY_WARPS * R * (32 / lpr);
-}
-
-template <int XMODE>
-static vq_status launch_moe_gemv(const MoeGemvArgs &a, int nproj, int max_active, cudaStream_t s)
+// Shared-memory plan and launch of moe_mma_kernel over the projections in m.
+static vq_status launch_moe_mma(MoeMmaArgs &m, cudaStream_t s)
 {
-    size_t smem = 0;
-    int gx = 1;
-    for (int z = 0; z < nproj; z++) {
-        smem = std::max(smem, cb_smem_bytes(a.W[z]));
-        const int rpc = gemv_rows_per_cta(a.W[z]);
-        gx = std::max(gx, (a.W[z].rows + rpc - 1) / rpc);
+    int64_t crb = 0, srow = 0;
+    int maxG = 1;
+    for (int p = 0; p < m.nproj; p++) {
+        crb = std::max(crb, m.W[p].code_row_bytes);
+        srow = std::max(srow, m.W[p].scale_row_elems * 2);
+        maxG = std::max(maxG, m.W[p].cols / 64);
+        if ((m.W[p].scale_row_elems * 2) % 16 || ((uintptr_t)m.W[p].scales % 16)) return VQ_ERR_UNSUPPORTED;
     }
-    auto kern = moe_gemv_kernel<XMODE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    m.NW = std::min(8, maxG);
+    m.slot_stride = (int)crb + 16;
+    m.stage_bytes = MMAV_ROWS * m.slot_stride + (int)((MMAV_ROWS * srow + 15) / 16 * 16);
+    const size_t fixed = 128 + SmemCB<8, 12>::BYTES + 2 * (size_t)m.NW * 16 * MMAV_ROWS * 4;
+    m.STAGES = 8;
+    while (m.STAGES > 2 && fixed + (size_t)m.STAGES * (m.stage_bytes + 16) > 232448) m.STAGES--;
+    const size_t smem = fixed + (size_t)m.STAGES * (m.stage_bytes + 16);
+    if (smem > 232448) return VQ_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(moe_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return VQ_ERR_CUDA;
-    dim3 grid(gx, max_active, nproj);
-    kern<<<grid, GEMV_BODY_THREADS, smem, s>>>(a);
+    moe_mma_kernel<<<moe_num_sms(), 32 * (1 + m.NW), smem, s>>>(m);
     VQ_CHECK_LAUNCH();
     return VQ_OK;
 }
@@ -382,9 +506,12 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     auto I = [&](size_t off) { return reinterpret_cast<int *>(W8 + off); };
     auto F = [&](size_t off) { return reinterpret_cast<float *>(W8 + off); };
 
-    // Tensor cores once experts see several tokens on average; the grouped GEMV otherwise.
+    // tcgen05 GEMM once experts see several tokens on average, or when a projection's
+    // scale rows are not whole 16-byte units (the tensor-core GEMV bulk-copies them);
+    // the grouped tensor-core GEMV otherwise.
     const double per_expert = (double)L.P / std::min(E, L.P);
-    const bool use_gemm = per_expert >= 4.0;
+    auto srows_ok = [](const Mat &M) { return (M.scale_row_elems * 2) % 16 == 0 && (uintptr_t)M.scales % 16 == 0; };
+    const bool use_gemm = per_expert >= 4.0 || !srows_ok(gate) || !srows_ok(up) || !srows_ok(down);
     const int BT = per_expert <= 24 ? 32 : per_expert <= 48 ? 64 : 128;
 
     BucketArgs b;
@@ -432,20 +559,39 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
         VQ_CHECK_LAUNCH();
         return VQ_OK;
     }
-    MoeGemvArgs a{};
-    a.sorted = b.sorted; a.offsets = b.offsets; a.act = b.act; a.nact = b.nact; a.topk = topk;
-    // gate and up in one grouped launch
-    a.W[0] = gate; a.W[1] = up;
-    a.out[0] = F(L.g); a.out[1] = F(L.u);
-    a.x = x;
-    st = xt == VQ_F16 ? launch_moe_gemv<0>(a, 2, max_active, s) : launch_moe_gemv<1>(a, 2, max_active, s);
-    if (st != VQ_OK) return st;
-    // down, input silu(g) * u
-    a.W[0] = down;
-    a.out[0] = F(L.o);
-    a.g = F(L.g); a.u = F(L.u);
-    if ((st = launch_moe_gemv<2>(a, 1, max_active, s)) != VQ_OK) return st;
-    // combine
+    // decode route: grouped tensor-core GEMV (tokens of an expert are the MMA's A rows)
+    const int64_t ng = (int64_t)L.P * (hidden / 8);
+    const __half *ain1 = static_cast<const __half *>(x);
+    int by_token = 1;
+    if (xt != VQ_F16) {   // bf16 activations: gather and convert to fp16 in bucket order
+        __half *xg = reinterpret_cast<__half *>(W8 + L.xg);
+        moe_gather_kernel<__nv_bfloat16><<<(unsigned)((ng + 255) / 256), 256, 0, s>>>(
+            (const __nv_bfloat16 *)x, b.sorted, b.offsets, E, topk, hidden, xg);
+        VQ_CHECK_LAUNCH();
+        ain1 = xg;
+        by_token = 0;
+    }
+    MoeMmaArgs m{};
+    m.sorted = b.sorted; m.offsets = b.offsets; m.act = b.act; m.nact = b.nact; m.topk = topk;
+    m.err = device_error_word();
+    if (!m.err) return VQ_ERR_CUDA;
+    m.nproj = 2;
+    m.W[0] = gate; m.W[1] = up;
+    m.out[0] = F(L.g); m.out[1] = F(L.u);
+    m.ain[0] = m.ain[1] = ain1;
+    m.a_by_token[0] = m.a_by_token[1] = by_token;
+    if ((st = launch_moe_mma(m, s)) != VQ_OK) return st;
+    __half *h16 = reinterpret_cast<__half *>(W8 + L.h16);
+    const int64_t nh = (int64_t)L.P * inter / 4;
+    moe_silu_mul_kernel<<<(unsigned)((nh + 255) / 256), 256, 0, s>>>(F(L.g), F(L.u), b.offsets, E, inter, h16);
+    VQ_CHECK_LAUNCH();
+    MoeMmaArgs md = m;
+    md.nproj = 1;
+    md.W[0] = down;
+    md.out[0] = F(L.o);
+    md.ain[0] = h16;
+    md.a_by_token[0] = 0;
+    if ((st = launch_moe_mma(md, s)) != VQ_OK) return st;
     const int64_t n = (int64_t)T * (hidden / 4);
     moe_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(F(L.o), b.pos, w, T, topk, hidden, y, (int)yt);
     VQ_CHECK_LAUNCH();
