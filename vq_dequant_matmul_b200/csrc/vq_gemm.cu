@@ -204,53 +204,66 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
         const uint8_t *cbl = sCB + (lane % CB::NREP) * CB::ENTRY;
         const uint32_t swz = (uint32_t)(t & 7);
 
-        Blk cur, nxt;
-        __half sc_cur = __float2half(0.f), sc_nxt = __float2half(0.f);
-        if (rv && par < nkb) { cur.load(crow, par); sc_cur = srow[par]; } else cur.zero();
-        for (int kb = par; kb < nkb; kb += 2) {
-            if (kb + 2 < nkb) {
-                if (rv) { nxt.load(crow, kb + 2); sc_nxt = srow[kb + 2]; } else nxt.zero();
-            }
-            const int s = kb % STAGES, r = kb / STAGES;
-            const bool ok = r == 0 || mbar_wait(&empty[s], (r - 1) & 1);
-            if (__any_sync(0xffffffffu, !ok || *abort_flag)) {   // warp-uniform exit
-                if (lane == 0) flag_error(abort_flag);
-                break;
-            }
-            const uint32_t arow = smem_u32(sA + s * A_TILE_BYTES) + t * 128;
-            const __half2 s2 = __half2half2(sc_cur);
-            const float sf = __half2float(sc_cur);
+        // Code blocks and scales of the stages kb = par + 2u (u < PF) are kept in flight in
+        // a register ring; a slot is refilled (PF stages ahead) right after it is expanded.
+        constexpr int PF = 3;
+        Blk ring[PF];
+        __half sr[PF];
 #pragma unroll
-            for (int c = 0; c < 8; c++) {
-                uint32_t o[4];
-                if constexpr (D == 2) {
+        for (int u = 0; u < PF; u++) {
+            const int kbu = par + 2 * u;
+            sr[u] = __float2half(0.f);
+            if (rv && kbu < nkb) { ring[u].load(crow, kbu); sr[u] = srow[kbu]; } else ring[u].zero();
+        }
+        bool stop = false;
+        for (int kb0 = par; kb0 < nkb && !stop; kb0 += 2 * PF) {
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        const uint32_t e = *reinterpret_cast<const uint32_t *>(cbl + cur.code(4 * c + j) * CB::STRIDE);
-                        o[j] = scale_pair<BF16T>(e, s2, sf);
-                    }
-                } else if constexpr (D == 4) {
-#pragma unroll
-                    for (int j = 0; j < 2; j++) {
-                        const uint2 e = *reinterpret_cast<const uint2 *>(cbl + cur.code(2 * c + j) * CB::STRIDE);
-                        o[2 * j] = scale_pair<BF16T>(e.x, s2, sf);
-                        o[2 * j + 1] = scale_pair<BF16T>(e.y, s2, sf);
-                    }
-                } else {
-                    const uint4 e = *reinterpret_cast<const uint4 *>(cbl + cur.code(c) * CB::STRIDE);
-                    o[0] = scale_pair<BF16T>(e.x, s2, sf);
-                    o[1] = scale_pair<BF16T>(e.y, s2, sf);
-                    o[2] = scale_pair<BF16T>(e.z, s2, sf);
-                    o[3] = scale_pair<BF16T>(e.w, s2, sf);
+            for (int u = 0; u < PF; u++) {
+                const int kb = kb0 + 2 * u;
+                if (kb >= nkb || stop) break;                       // uniform over the warp
+                const int s = kb % STAGES, r = kb / STAGES;
+                const bool ok = r == 0 || mbar_wait(&empty[s], (r - 1) & 1);
+                if (__any_sync(0xffffffffu, !ok || *abort_flag)) {   // warp-uniform exit
+                    if (lane == 0) flag_error(abort_flag);
+                    stop = true;
+                    break;
                 }
-                if (!rv) o[0] = o[1] = o[2] = o[3] = 0u;
-                sts128(arow + (((uint32_t)c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+                const uint32_t arow = smem_u32(sA + s * A_TILE_BYTES) + t * 128;
+                const __half2 s2 = __half2half2(sr[u]);
+                const float sf = __half2float(sr[u]);
+                const Blk &cur = ring[u];
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    uint32_t o[4];
+                    if constexpr (D == 2) {
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const uint32_t e = *reinterpret_cast<const uint32_t *>(cbl + cur.code(4 * c + j) * CB::STRIDE);
+                            o[j] = scale_pair<BF16T>(e, s2, sf);
+                        }
+                    } else if constexpr (D == 4) {
+#pragma unroll
+                        for (int j = 0; j < 2; j++) {
+                            const uint2 e = *reinterpret_cast<const uint2 *>(cbl + cur.code(2 * c + j) * CB::STRIDE);
+                            o[2 * j] = scale_pair<BF16T>(e.x, s2, sf);
+                            o[2 * j + 1] = scale_pair<BF16T>(e.y, s2, sf);
+                        }
+                    } else {
+                        const uint4 e = *reinterpret_cast<const uint4 *>(cbl + cur.code(c) * CB::STRIDE);
+                        o[0] = scale_pair<BF16T>(e.x, s2, sf);
+                        o[1] = scale_pair<BF16T>(e.y, s2, sf);
+                        o[2] = scale_pair<BF16T>(e.z, s2, sf);
+                        o[3] = scale_pair<BF16T>(e.w, s2, sf);
+                    }
+                    if (!rv) o[0] = o[1] = o[2] = o[3] = 0u;
+                    sts128(arow + (((uint32_t)c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_a[s]);
+                const int nk = kb + 2 * PF;                          // refill this slot
+                if (rv && nk < nkb) { ring[u].load(crow, nk); sr[u] = srow[nk]; }
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_a[s]);
-            cur = nxt;
-            sc_cur = sc_nxt;
         }
 
         // ---------------- epilogue: TMEM -> registers -> y
