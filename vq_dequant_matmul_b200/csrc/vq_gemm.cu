@@ -354,14 +354,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
+void *encode_tiled_fn();
+static EncodeTiledFn encode_fn() { return reinterpret_cast<EncodeTiledFn>(encode_tiled_fn()); }
+
+// cuTensorMapEncodeTiled from the driver (null if unavailable); shared with the GEMV.
+void *encode_tiled_fn() {
+    static void *fn = nullptr;
     if (!fn) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
+            fn = p;
     }
     return fn;
 }

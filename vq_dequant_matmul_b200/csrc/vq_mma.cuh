@@ -46,6 +46,50 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
     return v;
 }
 
+// Non-volatile forms for hot loops: the compiler may schedule them freely (overlapping
+// the latency of independent loads and MMAs), so their ordering against barriers must
+// come from data dependencies — addresses pass through launder() after the wait that
+// publishes the data, and results pass through consume() before the arrive that frees it.
+__device__ __forceinline__ uint32_t ldsn32(uint32_t a) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 ldsn64(uint32_t a) {
+    uint2 v;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 ldsn128(uint32_t a) {
+    uint4 v;
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t ldsn16(uint32_t a) {
+    unsigned short v;
+    asm("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void mman_f16_f32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mman_f16_f32_zero(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+// A value the compiler must treat as produced at this point of the program.
+__device__ __forceinline__ uint32_t launder(uint32_t v) {
+    asm volatile("" : "+r"(v)::"memory");
+    return v;
+}
+// A value the compiler must have computed by this point of the program.
+__device__ __forceinline__ void consume(float v) { asm volatile("" ::"f"(v) : "memory"); }
+
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar))
@@ -61,31 +105,34 @@ __device__ __forceinline__ void bar_arrive_named(int id, int nthreads) {
 }
 
 // The lane's codes of one scale group (64 columns) of its row, as they are needed by
-// the four MMAs: code(j) for j < 64 / d / 4.
-template <int D, int BITS>
+// the four MMAs: code(j) for j < 64 / d / 4.  NV: non-volatile loads (see ldsn32).
+template <int D, int BITS, bool NV = false>
 struct LaneCodes {
     uint32_t w0, w1, w2;
     int sh;   // 12-bit d = 4 / d = 8: bit offset inside w0:w1
+    static __device__ __forceinline__ uint32_t ld32(uint32_t a) { return NV ? ldsn32(a) : lds32(a); }
+    static __device__ __forceinline__ uint2 ld64(uint32_t a) { return NV ? ldsn64(a) : lds64(a); }
+    static __device__ __forceinline__ uint32_t ld16(uint32_t a) { return NV ? ldsn16(a) : lds16(a); }
     __device__ __forceinline__ void load(uint32_t grp_addr, int t) {
         if constexpr (BITS == 8) {
-            if constexpr (D == 2) { const uint2 v = lds64(grp_addr + 8 * t); w0 = v.x; w1 = v.y; }
-            else if constexpr (D == 4) { w0 = lds32(grp_addr + 4 * t); }
-            else { w0 = lds16(grp_addr + 2 * t); }
+            if constexpr (D == 2) { const uint2 v = ld64(grp_addr + 8 * t); w0 = v.x; w1 = v.y; }
+            else if constexpr (D == 4) { w0 = ld32(grp_addr + 4 * t); }
+            else { w0 = ld16(grp_addr + 2 * t); }
         } else {
             if constexpr (D == 2) {          // 12 bytes at 12t: codes at bits 12j
-                w0 = lds32(grp_addr + 12 * t);
-                w1 = lds32(grp_addr + 12 * t + 4);
-                w2 = lds32(grp_addr + 12 * t + 8);
+                w0 = ld32(grp_addr + 12 * t);
+                w1 = ld32(grp_addr + 12 * t + 4);
+                w2 = ld32(grp_addr + 12 * t + 8);
             } else if constexpr (D == 4) {   // 48 bits at bit 48t
                 const int wi = (3 * t) >> 1;
                 sh = 16 * (t & 1);
-                w0 = lds32(grp_addr + 4 * wi);
-                w1 = lds32(grp_addr + 4 * wi + 4);
+                w0 = ld32(grp_addr + 4 * wi);
+                w1 = ld32(grp_addr + 4 * wi + 4);
             } else {                         // 24 bits at bit 24t
                 const int bit = 24 * t;
                 sh = bit & 31;
-                w0 = lds32(grp_addr + 4 * (bit >> 5));
-                w1 = lds32(grp_addr + 4 * (bit >> 5) + 4);
+                w0 = ld32(grp_addr + 4 * (bit >> 5));
+                w1 = ld32(grp_addr + 4 * (bit >> 5) + 4);
             }
         }
     }
@@ -142,6 +189,12 @@ __device__ __forceinline__ void mma_group(uint32_t codes, int t, uint32_t cb_lan
 __device__ __forceinline__ void ldg_x16(const __half *p, uint32_t (&x)[8]) {
     const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
     const uint4 b = __ldg(reinterpret_cast<const uint4 *>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+__device__ __forceinline__ void ldsn_x16(uint32_t addr, uint32_t (&x)[8]) {
+    const uint4 a = ldsn128(addr);
+    const uint4 b = ldsn128(addr + 16);
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
