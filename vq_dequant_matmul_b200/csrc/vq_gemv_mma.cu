@@ -62,7 +62,7 @@ constexpr int GV_RB = 16;                    // weight rows per block (the MMA's
 template <int NT> __host__ __device__ constexpr int gv_nw() { return NT == 2 ? 8 : 16; }
 template <int NT> __host__ __device__ constexpr int gv_threads() { return 32 * (gv_nw<NT>() + 1); }
 constexpr int GV_MAX_STAGES = 10;
-constexpr int GV_MAX_R = GV_MAX_STAGES + 2;  // reduction buffers
+constexpr int GV_MAX_R = 14;                 // reduction buffers
 constexpr int GV_TBL = 65536;                // table region (64 KB)
 constexpr int GV_BAR_BYTES = 512;            // mbarriers + abort word
 constexpr int GV_DYN_SMEM = 232448;          // the per-block opt-in maximum (227 KB)
@@ -94,6 +94,7 @@ struct GvCfg {
     int XR, XB;        // staged activations: bytes per token row (0: read from global), total
     int PB;            // per-block results kept for the cluster reduction (0 if C = 1)
     int RBB;           // bytes of one reduction buffer
+    int lag;           // a block is reduced `lag` blocks after it is posted (so the wait is short)
     int CBB;           // bytes of the codebook as stored in global memory
     GvLayout L;
     unsigned int *err;
@@ -122,9 +123,9 @@ inline GvLayout gv_layout(const GvCfg &c, bool raw_cb) {
     L.ok = 0;
     const uint32_t a = (GV_LO + 1023u) & ~1023u, end = (uint32_t)GV_DYN_SMEM;
     for (int S = GV_MAX_STAGES; S >= 2; S--) {
-        // a warp can run S stages ahead of the slowest one; the reduction ring must cover
-        // that many row blocks plus the one being reduced
-        const int R = (S + 1 + c.nch - 1) / c.nch + 1;
+        // a warp can run S stages ahead of the slowest one, and a block is reduced `lag`
+        // blocks late: the reduction ring covers both, plus one spare
+        const int R = (S + 1 + c.nch - 1) / c.nch + c.lag + 1;
         GvBump r0{a, GV_TBL_ADDR}, r1{GV_TBL_ADDR + (uint32_t)GV_TBL, end};
         int n0 = (int)((GV_TBL_ADDR - a) / (uint32_t)c.SB);
         if (n0 > S) n0 = S;
@@ -446,8 +447,33 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
                                   (D == 2 ? (uint32_t)((t & 1) << 3) : D == 4 ? (uint32_t)(t << 2) : (uint32_t)(t << 1));
         const int nout = batch * GV_RB;
         float *const part = reinterpret_cast<float *>(sptr(A_part));
+        // sum block kb's partials over the warps, in warp order, and store (or keep) them
+        auto reduce = [&](int kb) -> bool {
+            const int rbk = kb % R;
+            const uint32_t rphk = (uint32_t)((kb / R) & 1);
+            const float *rbr = reinterpret_cast<const float *>(sptr(A_red + (uint32_t)(rbk * cfg.RBB)));
+            const bool ok = !aborted() && mbar_wait_sleep(&red_bar[rbk], rphk);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) fail();
+                return false;
+            }
+            for (int o = lane; o < nout; o += 32) {
+                float v = 0.f;
+#pragma unroll 4
+                for (int w = 0; w < NWK; w++) v += rbr[w * nout + o];
+                if (C == 1) {
+                    const int tok = o / GV_RB, r = (b0 + kb) * GV_RB + o % GV_RB;
+                    if (r < W.rows) store_out(y, (int64_t)tok * W.rows + r, v, yt);
+                } else if (q == 0) {
+                    part[kb * nout + o] = v;
+                } else {   // straight into rank 0's receive buffer
+                    st_cluster_f32(A_recv + (uint32_t)(((q - 1) * nb * nout + kb * nout + o) * 4), 0u, v);
+                }
+            }
+            return true;
+        };
         int slot = 0, rbi = 0;
-        uint32_t ph = 0, rph = 0;
+        uint32_t ph = 0;
         for (int kb = 0; kb < nb && !stop; kb++) {
             float acc[NT][4];
 #pragma unroll
@@ -557,30 +583,16 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
                 ua = ue;
             }
             if (stop) break;
-            if ((kb & (NWK - 1)) == cw) {
-                // reduce block kb over the warps, in warp order
-                const bool ok = !aborted() && mbar_wait_sleep(&red_bar[rbi], rph);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0) fail();
-                    stop = true;
-                    break;
-                }
-                for (int o = lane; o < nout; o += 32) {
-                    float v = 0.f;
-#pragma unroll 4
-                    for (int w = 0; w < NWK; w++) v += rb[w * nout + o];
-                    if (C == 1) {
-                        const int tok = o / GV_RB, r = (b0 + kb) * GV_RB + o % GV_RB;
-                        if (r < W.rows) store_out(y, (int64_t)tok * W.rows + r, v, yt);
-                    } else if (q == 0) {
-                        part[kb * nout + o] = v;
-                    } else {   // straight into rank 0's receive buffer
-                        st_cluster_f32(A_recv + (uint32_t)(((q - 1) * nb * nout + kb * nout + o) * 4), 0u, v);
-                    }
-                }
+            // reduce block kb - lag (posted long enough ago that the wait is short)
+            if (kb >= cfg.lag && ((kb - cfg.lag) & (NWK - 1)) == cw && !reduce(kb - cfg.lag)) {
+                stop = true;
+                break;
             }
-            if (++rbi == R) { rbi = 0; rph ^= 1u; }
+            if (++rbi == R) rbi = 0;
         }
+        // the last `lag` blocks
+        for (int kb = max(0, nb - cfg.lag); kb < nb && !stop; kb++)
+            if ((kb & (NWK - 1)) == cw && !reduce(kb)) stop = true;
     }
 
     if (C > 1) {
@@ -789,6 +801,7 @@ vq_status gv_launch5(const Mat &W, const void *x, int batch, void *y, int yt, Gv
         c.XB = XS ? batch * c.XR : 0;
         c.PB = c.C > 1 ? bpc * batch * GV_RB * 4 : 0;
         c.RBB = gv_nw<NT>() * batch * GV_RB * 4;
+        c.lag = NT == 1 ? 2 : 0;   // (batches 9..16: buffers too large for a longer ring)
         c.CBB = (1 << BITS) * D * 2;
         c.L = gv_layout(c, BITS == 8);
         fits = c.L.ok && c.L.stages >= 3;
