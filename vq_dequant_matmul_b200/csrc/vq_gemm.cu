@@ -14,11 +14,15 @@
 //   * warps 2-9 (256 threads, two per weight row, taking alternate 64-column stages, so
 //     each thread's code prefetch runs two stages ahead) read the row's packed codes and
 //     scale straight from global memory, look the codes up in the shared-memory
-//     codebook, multiply by the scale (one rounding to the tile type) and write the
-//     128 x 64 tile in the same 128-byte-swizzled K-major layout, then fence the
-//     generic->async proxy and signal an mbarrier;
-//   * warp 1 (one thread) issues tcgen05.mma (kind::f16, fp32 accumulation in tensor
-//     memory) for each 64-column stage and frees the stage with tcgen05.commit;
+//     codebook and multiply by the scale (one rounding to the tile type).  The expanded
+//     128 x 64 tile goes to tensor memory: each thread writes its row (a warp may only
+//     reach its own 32-lane quarter, so row = 32 (warp mod 4) + lane) as 32 columns with
+//     one tcgen05.st, then signals an mbarrier.  Keeping the A tile out of shared memory
+//     leaves the shared-memory bandwidth to the codebook lookups and the activation
+//     tiles, which the MMA reads from there;
+//   * warp 1 (one thread) issues tcgen05.mma (kind::f16, A from tensor memory, B from
+//     shared memory, fp32 accumulation in tensor memory) for each 64-column stage and
+//     frees the stage with tcgen05.commit;
 //   * after the last stage, warps 2-9 read the accumulator out of tensor memory
 //     (tcgen05.ld; two warps per 32-lane quarter, each half of the columns) and store y.
 // Stages are a ring of STAGES buffers guarded by mbarriers; every wait is bounded and a
@@ -37,7 +41,6 @@ __device__ unsigned int g_device_error;   // nonzero after a bounded wait ran ou
 constexpr int GEMM_BM = 128;       // weight rows per tile (UMMA M)
 constexpr int GEMM_BK = 64;        // columns per stage (one 128-byte swizzle row of 16-bit)
 constexpr int GEMM_THREADS = 320;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 expansion + epilogue
-constexpr int A_TILE_BYTES = GEMM_BM * GEMM_BK * 2;
 
 // Packed codes of one row for one 64-column stage: 64/d codes.
 template <int D, int BITS>
@@ -93,11 +96,6 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t cb2, __half2 s2, float s
     }
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
-
 __device__ __forceinline__ void flag_error(volatile int *abort_flag) {
     *abort_flag = 1;
     atomicExch(&g_device_error, 1u);
@@ -112,11 +110,15 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
     using CB = SmemCB<D, BITS>;
     using Blk = CodeBlock<D, BITS>;
     constexpr int B_TILE_BYTES = BT * GEMM_BK * 2;
-    constexpr uint32_t TMEM_COLS = BT;          // fp32 accumulator: one column per token
+    // tensor memory: fp32 accumulator (one column per token), then one 32-column A tile
+    // per stage; the allocation is a power of two
+    constexpr uint32_t TMEM_NEED = BT + 32 * STAGES;
+    constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                   : TMEM_NEED <= 256 ? 256 : 512;
+    static_assert(TMEM_NEED <= 512, "tensor memory holds 512 columns");
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;
-    uint8_t *sB = sA + STAGES * A_TILE_BYTES;
+    uint8_t *sB = smem;
     uint8_t *sCB = sB + STAGES * B_TILE_BYTES;
     uint64_t *full_a = reinterpret_cast<uint64_t *>(sCB + CB::BYTES);
     uint64_t *full_b = full_a + STAGES;
@@ -182,11 +184,11 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
                     break;
                 }
                 tc_fence_after();
-                const uint64_t adesc = smem_desc_sw128(smem_u32(sA + s * A_TILE_BYTES));
                 const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * B_TILE_BYTES));
 #pragma unroll
-                for (int k = 0; k < GEMM_BK / 16; k++)   // K = 16 per MMA: +32 bytes = +2 in the address field
-                    umma_f16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                for (int k = 0; k < GEMM_BK / 16; k++)   // K = 16 per MMA: 8 A columns; +32 bytes = +2 in B's address field
+                    umma_f16_ts(tmem, tmem + (uint32_t)(BT + 32 * s + 8 * k), bdesc + 2 * k, idesc,
+                                (kb > 0 || k > 0) ? 1u : 0u);
                 umma_commit(&empty[s]);
                 *consumed = kb + 1;
             }
@@ -194,15 +196,14 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
         }
     } else {
         // ---------------- expansion: thread t writes weight row n0 + t of every stage
-        const int et = threadIdx.x - 64;
-        const int t = et & (GEMM_BM - 1);        // tile row
-        const int par = et >> 7;                 // this thread expands stages kb = par, par + 2, ...
+        const int t = 32 * (warp & 3) + lane;    // tile row = tensor-memory lane
+        const int par = (warp - 2) >> 2;         // this thread expands stages kb = par, par + 2, ...
         const int row = n0 + t;
         const bool rv = row < W.rows;
         const uint8_t *crow = codes_e + (int64_t)(rv ? row : 0) * W.code_row_bytes;
         const __half *srow = scales_e + (int64_t)(rv ? row : 0) * W.scale_row_elems;
         const uint8_t *cbl = sCB + (lane % CB::NREP) * CB::ENTRY;
-        const uint32_t swz = (uint32_t)(t & 7);
+        const uint32_t tquarter = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's tensor-memory lanes
 
         // Code blocks and scales of the stages kb = par + 2u (u < PF) are kept in flight in
         // a register ring; a slot is refilled (PF stages ahead) right after it is expanded.
@@ -228,7 +229,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
                     stop = true;
                     break;
                 }
-                const uint32_t arow = smem_u32(sA + s * A_TILE_BYTES) + t * 128;
+                uint32_t av[32];                                     // the row's 64 tile elements
                 const __half2 s2 = __half2half2(sr[u]);
                 const float sf = __half2float(sr[u]);
                 const Blk &cur = ring[u];
@@ -256,9 +257,12 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
                         o[3] = scale_pair<BF16T>(e.w, s2, sf);
                     }
                     if (!rv) o[0] = o[1] = o[2] = o[3] = 0u;
-                    sts128(arow + (((uint32_t)c ^ swz) << 4), o[0], o[1], o[2], o[3]);
+#pragma unroll
+                    for (int j = 0; j < 4; j++) av[4 * c + j] = o[j];   // column 4c + j: elements 8c + 2j, +1
                 }
-                fence_proxy_async_smem();
+                tmem_st_32x32b_x32(tmem + tquarter + (uint32_t)(BT + 32 * s), av);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_a[s]);
                 const int nk = kb + 2 * PF;                          // refill this slot
@@ -387,7 +391,7 @@ static bool make_x_map(CUtensorMap *map, const void *x, bool bf16, int M, int K,
 
 // Shared memory of a launch whose largest codebook table takes cb_bytes.
 static size_t gemm_smem_bytes(int BT, int stages, size_t cb_bytes) {
-    return 1024 + (size_t)stages * (A_TILE_BYTES + (size_t)BT * GEMM_BK * 2) + cb_bytes + (3 * stages + 1) * 8 + 16;
+    return 1024 + (size_t)stages * ((size_t)BT * GEMM_BK * 2) + cb_bytes + (3 * stages + 1) * 8 + 16;
 }
 
 static size_t cb_table_bytes(const Mat &W) {
@@ -421,6 +425,8 @@ static vq_status launch_gemm_bt(const CUtensorMap &map, const GemmArgs &a, int n
 {
     size_t cb = 0;
     for (int z = 0; z < nproj; z++) cb = std::max(cb, cb_table_bytes(a.W[z]));
+    if (BT + 32 * 6 <= 512 && gemm_smem_bytes(BT, 6, cb) <= 232448)
+        return launch_gemm_cfg<BT, 6, BF16T>(map, a, nproj, gx, gemm_smem_bytes(BT, 6, cb), s);
     if (gemm_smem_bytes(BT, 4, cb) <= 232448)
         return launch_gemm_cfg<BT, 4, BF16T>(map, a, nproj, gx, gemm_smem_bytes(BT, 4, cb), s);
     if (gemm_smem_bytes(BT, 3, cb) <= 232448)

@@ -205,7 +205,9 @@ struct MoeMmaArgs {
     int a_by_token[3];
     const int *sorted, *offsets, *act, *nact;
     int topk;
-    int NW, STAGES, slot_stride, stage_bytes;
+    int NW, STAGES, stage_bytes, soff;
+    int tbl_off[3];              // shared-memory offset of each projection's codebook table
+    int tbl_bytes;
     unsigned int *err;
 };
 
@@ -228,49 +230,74 @@ __device__ __forceinline__ MoeItem moe_item(const MoeMmaArgs &a, int i, int nact
     return it;
 }
 
+// One item (an 8-row block of one expert's projection) by one warp: every scale group,
+// every token of the expert (16 per pass: the MMA's A rows g and g + 8), and the
+// outputs of its 8 rows.  `stage` holds the block's rows (code_row_bytes apart) and, at
+// `sc`, their scales.
 template <int D, int BITS>
-__device__ __forceinline__ void moe_mma_chunk(const MoeMmaArgs &a, const Mat &W, int p, uint32_t stage,
-                                              uint32_t cb_lane, int cw, int lane, int c0, int j1, float (&tot)[2][2])
+__device__ __forceinline__ void moe_warp_item(const MoeMmaArgs &a, const Mat &W, int p, uint32_t stage, uint32_t sc,
+                                              uint32_t cb_lane, int lane, int j0, int j1, int r0)
 {
     constexpr int GB = (64 / D) * BITS / 8;
     const int g = lane >> 2, t = lane & 3;
     const int G = W.cols / 64;
-    const int pos0 = min(c0 + g, j1 - 1), pos1 = min(c0 + g + 8, j1 - 1);
-    const __half *r0, *r1;
-    if (a.a_by_token[p]) {
-        r0 = a.ain[p] + (int64_t)(a.sorted[pos0] / a.topk) * W.cols;
-        r1 = a.ain[p] + (int64_t)(a.sorted[pos1] / a.topk) * W.cols;
-    } else {
-        r0 = a.ain[p] + (int64_t)pos0 * W.cols;
-        r1 = a.ain[p] + (int64_t)pos1 * W.cols;
-    }
-    r0 += 16 * t;
-    r1 += 16 * t;
-    const uint32_t row_lane = stage + g * a.slot_stride;
-    const uint32_t sc_base = stage + MMAV_ROWS * a.slot_stride;
-    for (int grp = cw; grp < G; grp += a.NW) {
-        uint32_t x0[8], x1[8];
-        ldg_x16(r0 + grp * 64, x0);
-        ldg_x16(r1 + grp * 64, x1);
-        float d[4];
-        mma_group<D, BITS>(row_lane + grp * GB, t, cb_lane, x0, x1, d);
-        const float s0 = __half2float(__ushort_as_half((unsigned short)lds16(sc_base + ((2 * t) * (int)W.scale_row_elems + grp) * 2)));
-        const float s1 = __half2float(__ushort_as_half((unsigned short)lds16(sc_base + ((2 * t + 1) * (int)W.scale_row_elems + grp) * 2)));
-        tot[0][0] = fmaf(s0, d[0], tot[0][0]);
-        tot[0][1] = fmaf(s1, d[1], tot[0][1]);
-        tot[1][0] = fmaf(s0, d[2], tot[1][0]);
-        tot[1][1] = fmaf(s1, d[3], tot[1][1]);
+    const uint32_t crb = (uint32_t)W.code_row_bytes, srow = (uint32_t)W.scale_row_elems * 2;
+    const uint32_t row_lane = stage + (uint32_t)g * crb;
+    const uint32_t sc0 = sc + (uint32_t)(2 * t) * srow, sc1 = sc0 + srow;   // scales of rows 2t, 2t + 1
+    for (int c0 = j0; c0 < j1; c0 += 16) {
+        const int pos0 = min(c0 + g, j1 - 1), pos1 = min(c0 + g + 8, j1 - 1);
+        const __half *x0p, *x1p;
+        if (a.a_by_token[p]) {
+            x0p = a.ain[p] + (int64_t)(a.sorted[pos0] / a.topk) * W.cols;
+            x1p = a.ain[p] + (int64_t)(a.sorted[pos1] / a.topk) * W.cols;
+        } else {
+            x0p = a.ain[p] + (int64_t)pos0 * W.cols;
+            x1p = a.ain[p] + (int64_t)pos1 * W.cols;
+        }
+        x0p += 16 * t;
+        x1p += 16 * t;
+        float tot[2][2] = {{0.f, 0.f}, {0.f, 0.f}};   // [token g / g + 8][row 2t / 2t + 1]
+        for (int grp = 0; grp < G; grp++) {
+            uint32_t xa[8], xb[8];
+            ldg_x16(x0p + grp * 64, xa);
+            ldg_x16(x1p + grp * 64, xb);
+            float d[4];
+            mma_group<D, BITS>(row_lane + (uint32_t)(grp * GB), t, cb_lane, xa, xb, d);
+            const float s0 = __half2float(__ushort_as_half((unsigned short)lds16(sc0 + 2u * grp)));
+            const float s1 = __half2float(__ushort_as_half((unsigned short)lds16(sc1 + 2u * grp)));
+            tot[0][0] = fmaf(s0, d[0], tot[0][0]);
+            tot[0][1] = fmaf(s1, d[1], tot[0][1]);
+            tot[1][0] = fmaf(s0, d[2], tot[1][0]);
+            tot[1][1] = fmaf(s1, d[3], tot[1][1]);
+        }
+        float *out = a.out[p];
+        const int ra = r0 + 2 * t, rb = ra + 1;
+        if (c0 + g < j1) {
+            if (ra < W.rows) out[(int64_t)(c0 + g) * W.rows + ra] = tot[0][0];
+            if (rb < W.rows) out[(int64_t)(c0 + g) * W.rows + rb] = tot[0][1];
+        }
+        if (c0 + g + 8 < j1) {
+            if (ra < W.rows) out[(int64_t)(c0 + g + 8) * W.rows + ra] = tot[1][0];
+            if (rb < W.rows) out[(int64_t)(c0 + g + 8) * W.rows + rb] = tot[1][1];
+        }
     }
 }
 
+// Grouped tensor-core GEMV over (projection, active expert, 8-row block) items.  Each CTA
+// takes a balanced contiguous range of items.  Warp 0 (one thread) streams each item's
+// rows and scales into a ring of stages with two bulk copies (an expert's rows are
+// contiguous) and writes the expert's bucket range [j0, j1) into the stage's header;
+// consumer warp w takes items w, w + NW, ..., so the CTA works on NW items at once and no
+// warp waits for another.  Every projection's codebook table stays resident (projections
+// of one launch may be in flight together), so experts must share their tensor's
+// codebook on this path.
 __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    uint8_t *sCB = smem;
-    uint8_t *sStage = sCB + SmemCB<8, 12>::BYTES;            // largest table (64 KB)
-    float *red = reinterpret_cast<float *>(sStage + (size_t)a.STAGES * a.stage_bytes);   // [2][NW][16][8]
-    uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * a.NW * 16 * MMAV_ROWS);
+    uint8_t *sStage = smem + a.tbl_bytes;
+    int2 *hdr = reinterpret_cast<int2 *>(sStage + (size_t)a.STAGES * a.stage_bytes);   // [STAGES]
+    uint64_t *full = reinterpret_cast<uint64_t *>(hdr + a.STAGES);
     uint64_t *empty = full + a.STAGES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -284,7 +311,7 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.STAGES; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], a.NW);
+            mbar_init(&empty[s], 1);
         }
         mbar_fence_init();
     }
@@ -302,90 +329,68 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
                 const Mat &W = a.W[it.p];
                 const int r0 = it.blk * MMAV_ROWS;
                 const int nrows = min(MMAV_ROWS, W.rows - r0);
-                const uint8_t *codes = W.codes + (int64_t)it.e * W.expert_code_stride;
-                const __half *scales = W.scales + (int64_t)it.e * W.expert_scale_stride;
+                const uint8_t *codes = W.codes + (int64_t)it.e * W.expert_code_stride + (int64_t)r0 * W.code_row_bytes;
+                const __half *scales = W.scales + (int64_t)it.e * W.expert_scale_stride + (int64_t)r0 * W.scale_row_elems;
+                hdr[slot] = make_int2(a.offsets[it.e], a.offsets[it.e + 1]);   // published by the arrive below
                 const uint32_t base = smem_u32(sStage + (size_t)slot * a.stage_bytes);
-                mbar_arrive_expect_tx(&full[slot], (uint32_t)(nrows * (W.code_row_bytes + W.scale_row_elems * 2)));
-                for (int r = 0; r < nrows; r++)
-                    bulk_copy_g2s(base + r * a.slot_stride, codes + (int64_t)(r0 + r) * W.code_row_bytes,
-                                  (uint32_t)W.code_row_bytes, &full[slot]);
-                bulk_copy_g2s(base + MMAV_ROWS * a.slot_stride, scales + (int64_t)r0 * W.scale_row_elems,
-                              (uint32_t)(nrows * W.scale_row_elems * 2), &full[slot]);
+                const uint32_t cbytes = (uint32_t)(nrows * W.code_row_bytes);
+                const uint32_t sbytes = (uint32_t)(nrows * W.scale_row_elems * 2);
+                mbar_arrive_expect_tx(&full[slot], cbytes + sbytes);
+                bulk_copy_g2s(base, codes, cbytes, &full[slot]);
+                bulk_copy_g2s(base + (uint32_t)a.soff, scales, sbytes, &full[slot]);
             }
         }
         return;
     }
 
+    // every projection's codebook table
+    const int nthr = a.NW * 32, ctid = threadIdx.x - 32;
+    for (int p = 0; p < a.nproj; p++) {
+        uint8_t *tb = smem + a.tbl_off[p];
+        const __half *cb = a.W[p].codebook;
+        switch (geom_of(a.W[p].d, a.W[p].bits)) {
+        case G_D2_B8: SmemCB<2, 8>::stage(tb, cb, ctid, nthr); break;
+        case G_D4_B8: SmemCB<4, 8>::stage(tb, cb, ctid, nthr); break;
+        case G_D8_B8: SmemCB<8, 8>::stage(tb, cb, ctid, nthr); break;
+        case G_D2_B12: SmemCB<2, 12>::stage(tb, cb, ctid, nthr); break;
+        case G_D4_B12: SmemCB<4, 12>::stage(tb, cb, ctid, nthr); break;
+        default: SmemCB<8, 12>::stage(tb, cb, ctid, nthr); break;
+        }
+    }
+    bar_sync_named(1, nthr);
+
     const int cw = warp - 1;
-    const int nthr = a.NW * 32;
-    const __half *cur_cb = nullptr;
-    bool dead = false;
-    int rbuf = 0;
-    for (int i = i_begin, k = 0; i < i_end; i++, k++) {
+    for (int i = i_begin + cw, k = cw; i < i_end; i += a.NW, k += a.NW) {
         const int slot = k % a.STAGES, round = k / a.STAGES;
+        const bool ok = mbar_wait(&full[slot], round & 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+            if (lane == 0) atomicExch(a.err, 1u);
+            break;
+        }
         const MoeItem it = moe_item(a, i, nact);
         const Mat &W = a.W[it.p];
-        const int geom = geom_of(W.d, W.bits);
-        const __half *cb = W.codebook + (int64_t)it.e * W.expert_codebook_stride;
-        if (cb != cur_cb) {                                     // (re)stage the codebook
-            bar_sync_named(1, nthr);
-            switch (geom) {
-            case G_D2_B8: SmemCB<2, 8>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
-            case G_D4_B8: SmemCB<4, 8>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
-            case G_D8_B8: SmemCB<8, 8>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
-            case G_D2_B12: SmemCB<2, 12>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
-            case G_D4_B12: SmemCB<4, 12>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
-            default: SmemCB<8, 12>::stage(sCB, cb, threadIdx.x - 32, nthr); break;
-            }
-            bar_sync_named(1, nthr);
-            cur_cb = cb;
-        }
-        if (!dead) {
-            const bool ok = mbar_wait(&full[slot], round & 1);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) atomicExch(a.err, 1u);
-                dead = true;
-            }
-        }
+        const int2 jj = hdr[slot];
         const uint32_t stage = smem_u32(sStage + (size_t)slot * a.stage_bytes);
-        const int j0 = a.offsets[it.e], j1 = a.offsets[it.e + 1];
+        const uint32_t tbl = smem_u32(smem + a.tbl_off[it.p]);
         const int r0 = it.blk * MMAV_ROWS;
-        for (int c0 = j0; c0 < j1; c0 += 16) {
-            float tot[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-            if (!dead) {
-                switch (geom) {
-#define VQ_MOE_CASE(GG, DD, BB)                                                                              \
-    case GG: moe_mma_chunk<DD, BB>(a, W, it.p, stage, smem_u32(sCB) + (lane % SmemCB<DD, BB>::NREP) *       \
-                                   SmemCB<DD, BB>::ENTRY, cw, lane, c0, j1, tot); break;
-                VQ_MOE_CASE(G_D2_B8, 2, 8)
-                VQ_MOE_CASE(G_D4_B8, 4, 8)
-                VQ_MOE_CASE(G_D8_B8, 8, 8)
-                VQ_MOE_CASE(G_D2_B12, 2, 12)
-                VQ_MOE_CASE(G_D4_B12, 4, 12)
-                VQ_MOE_CASE(G_D8_B12, 8, 12)
+        switch (geom_of(W.d, W.bits)) {
+#define VQ_MOE_CASE(GG, DD, BB)                                                                                  \
+    case GG:                                                                                                   \
+        moe_warp_item<DD, BB>(a, W, it.p, stage, stage + (uint32_t)a.soff,                                     \
+                              tbl + (uint32_t)((lane % SmemCB<DD, BB>::NREP) * SmemCB<DD, BB>::ENTRY), lane,   \
+                              jj.x, jj.y, r0);                                                                 \
+        break;
+        VQ_MOE_CASE(G_D2_B8, 2, 8)
+        VQ_MOE_CASE(G_D4_B8, 4, 8)
+        VQ_MOE_CASE(G_D8_B8, 8, 8)
+        VQ_MOE_CASE(G_D2_B12, 2, 12)
+        VQ_MOE_CASE(G_D4_B12, 4, 12)
+        VQ_MOE_CASE(G_D8_B12, 8, 12)
 #undef VQ_MOE_CASE
-                default: break;
-                }
-            }
-            if (c0 + 16 >= j1) {                                // last read of this stage
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[slot]);
-            }
-            float *rb = red + rbuf * a.NW * 16 * MMAV_ROWS;
-            const int g = lane >> 2, t = lane & 3;
-            rb[(cw * 16 + g) * MMAV_ROWS + 2 * t] = tot[0][0];
-            rb[(cw * 16 + g) * MMAV_ROWS + 2 * t + 1] = tot[0][1];
-            rb[(cw * 16 + g + 8) * MMAV_ROWS + 2 * t] = tot[1][0];
-            rb[(cw * 16 + g + 8) * MMAV_ROWS + 2 * t + 1] = tot[1][1];
-            bar_sync_named(1, nthr);
-            for (int q = cw * 32 + lane; q < 16 * MMAV_ROWS; q += nthr) {
-                const int tk = q / MMAV_ROWS, rr = q % MMAV_ROWS;
-                float v = 0.f;
-                for (int w = 0; w < a.NW; w++) v += rb[(w * 16 + tk) * MMAV_ROWS + rr];
-                if (c0 + tk < j1 && r0 + rr < W.rows) a.out[it.p][(int64_t)(c0 + tk) * W.rows + r0 + rr] = v;
-            }
-            rbuf ^= 1;
+        default: break;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
     }
 }
 
@@ -469,24 +474,42 @@ static int moe_num_sms() {
     return n > 0 ? n : 148;
 }
 
-// Shared-memory plan and launch of moe_mma_kernel over the projections in m.
+// Shared-memory plan and launch of moe_mma_kernel over the projections in m:
+// UNSUPPORTED (nothing launched) when the tables and a ring of at least 2 * NW stages do
+// not fit, or a projection's scale rows are not whole 16-byte units.
+static size_t moe_table_bytes(const Mat &W) {
+    switch (geom_of(W.d, W.bits)) {
+    case G_D2_B8: return SmemCB<2, 8>::BYTES;
+    case G_D4_B8: return SmemCB<4, 8>::BYTES;
+    case G_D8_B8: return SmemCB<8, 8>::BYTES;
+    case G_D2_B12: return SmemCB<2, 12>::BYTES;
+    case G_D4_B12: return SmemCB<4, 12>::BYTES;
+    default: return SmemCB<8, 12>::BYTES;
+    }
+}
+
 static vq_status launch_moe_mma(MoeMmaArgs &m, cudaStream_t s)
 {
     int64_t crb = 0, srow = 0;
-    int maxG = 1;
+    size_t tb = 0;
     for (int p = 0; p < m.nproj; p++) {
         crb = std::max(crb, m.W[p].code_row_bytes);
         srow = std::max(srow, m.W[p].scale_row_elems * 2);
-        maxG = std::max(maxG, m.W[p].cols / 64);
         if ((m.W[p].scale_row_elems * 2) % 16 || ((uintptr_t)m.W[p].scales % 16)) return VQ_ERR_UNSUPPORTED;
+        if (m.W[p].num_experts > 1 && (m.W[p].expert_scale_stride * 2) % 16) return VQ_ERR_UNSUPPORTED;
+        if (m.W[p].num_experts > 1 && m.W[p].expert_codebook_stride != 0) return VQ_ERR_UNSUPPORTED;
+        m.tbl_off[p] = (int)tb;
+        tb += (moe_table_bytes(m.W[p]) + 127) / 128 * 128;
     }
-    m.NW = std::min(8, maxG);
-    m.slot_stride = (int)crb + 16;
-    m.stage_bytes = MMAV_ROWS * m.slot_stride + (int)((MMAV_ROWS * srow + 15) / 16 * 16);
-    const size_t fixed = 128 + SmemCB<8, 12>::BYTES + 2 * (size_t)m.NW * 16 * MMAV_ROWS * 4;
-    m.STAGES = 8;
-    while (m.STAGES > 2 && fixed + (size_t)m.STAGES * (m.stage_bytes + 16) > 232448) m.STAGES--;
-    const size_t smem = fixed + (size_t)m.STAGES * (m.stage_bytes + 16);
+    m.tbl_bytes = (int)tb;
+    m.NW = 8;
+    m.soff = (int)(MMAV_ROWS * crb);
+    m.stage_bytes = (int)((MMAV_ROWS * crb + MMAV_ROWS * srow + 127) / 128 * 128);
+    const size_t fixed = 128 + tb;
+    const size_t per_stage = (size_t)m.stage_bytes + sizeof(int2) + 16;
+    m.STAGES = 32;
+    while (m.STAGES > 2 * m.NW && fixed + (size_t)m.STAGES * per_stage > 232448) m.STAGES--;
+    const size_t smem = fixed + (size_t)m.STAGES * per_stage;
     if (smem > 232448) return VQ_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(moe_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return VQ_ERR_CUDA;
@@ -506,12 +529,18 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     auto I = [&](size_t off) { return reinterpret_cast<int *>(W8 + off); };
     auto F = [&](size_t off) { return reinterpret_cast<float *>(W8 + off); };
 
-    // tcgen05 GEMM once experts see several tokens on average, or when a projection's
-    // scale rows are not whole 16-byte units (the tensor-core GEMV bulk-copies them);
-    // the grouped tensor-core GEMV otherwise.
+    // tcgen05 GEMM once experts see several tokens on average, when a projection's scale
+    // rows are not whole 16-byte units (the tensor-core GEMV bulk-copies them), or when
+    // experts have codebooks of their own (the GEMV keeps one table per projection); the
+    // grouped tensor-core GEMV otherwise.
     const double per_expert = (double)L.P / std::min(E, L.P);
-    auto srows_ok = [](const Mat &M) { return (M.scale_row_elems * 2) % 16 == 0 && (uintptr_t)M.scales % 16 == 0; };
-    const bool use_gemm = per_expert >= 4.0 || !srows_ok(gate) || !srows_ok(up) || !srows_ok(down);
+    auto srows_ok = [](const Mat &M) {
+        return (M.scale_row_elems * 2) % 16 == 0 && (uintptr_t)M.scales % 16 == 0 &&
+               (M.num_experts == 1 || (M.expert_scale_stride * 2) % 16 == 0);
+    };
+    auto shared_cb = [](const Mat &M) { return M.num_experts == 1 || M.expert_codebook_stride == 0; };
+    const bool use_gemm = per_expert >= 4.0 || !srows_ok(gate) || !srows_ok(up) || !srows_ok(down) ||
+                          !shared_cb(gate) || !shared_cb(up) || !shared_cb(down);
     const int BT = per_expert <= 24 ? 32 : per_expert <= 48 ? 64 : 128;
 
     BucketArgs b;
