@@ -12,7 +12,7 @@
 //   * warp 0 (one thread) streams activation tiles [BT][64] into shared memory with TMA
 //     (128-byte swizzle);
 //   * warps 2-9 (256 threads, two per weight row, taking alternate 64-column stages, so
-//     each thread's code prefetch runs two stages ahead) read the row's packed codes and
+//     each thread's code prefetch runs several stages ahead) read the row's packed codes and
 //     scale straight from global memory, look the codes up in the shared-memory
 //     codebook and multiply by the scale (one rounding to the tile type).  The expanded
 //     128 x 64 tile goes to tensor memory: each thread writes its row (a warp may only
@@ -207,7 +207,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
 
         // Code blocks and scales of the stages kb = par + 2u (u < PF) are kept in flight in
         // a register ring; a slot is refilled (PF stages ahead) right after it is expanded.
-        constexpr int PF = 3;
+        constexpr int PF = 5;
         Blk ring[PF];
         __half sr[PF];
 #pragma unroll

@@ -162,26 +162,28 @@ template <int D, int BITS>
 __device__ __forceinline__ void mma_group(uint32_t codes, int t, uint32_t cb_lane, const uint32_t (&xa)[8],
                                           const uint32_t (&xb)[8], float (&d)[4])
 {
+    // non-volatile loads and MMAs (see ldsn32): `codes` must come from a laundered stage
+    // address and `cb_lane` from a laundered table address
     using CB = SmemCB<D, BITS>;
-    LaneCodes<D, BITS> lc;
+    LaneCodes<D, BITS, true> lc;
     lc.load(codes, t);
-    d[0] = d[1] = d[2] = d[3] = 0.f;
 #pragma unroll
     for (int s = 0; s < 4; s++) {
         const uint32_t a[4] = {xa[2 * s], xb[2 * s], xa[2 * s + 1], xb[2 * s + 1]};
         uint32_t b0, b1;
         if constexpr (D == 2) {
-            b0 = lds32(cb_lane + lc.code(2 * s) * CB::STRIDE);
-            b1 = lds32(cb_lane + lc.code(2 * s + 1) * CB::STRIDE);
+            b0 = ldsn32(cb_lane + lc.code(2 * s) * CB::STRIDE);
+            b1 = ldsn32(cb_lane + lc.code(2 * s + 1) * CB::STRIDE);
         } else if constexpr (D == 4) {
-            const uint2 e = lds64(cb_lane + lc.code(s) * CB::STRIDE);
+            const uint2 e = ldsn64(cb_lane + lc.code(s) * CB::STRIDE);
             b0 = e.x; b1 = e.y;
         } else {
-            const uint4 e = lds128(cb_lane + lc.code(s >> 1) * CB::STRIDE);
+            const uint4 e = ldsn128(cb_lane + lc.code(s >> 1) * CB::STRIDE);
             b0 = (s & 1) ? e.z : e.x;
             b1 = (s & 1) ? e.w : e.y;
         }
-        mma_f16_f32(d, a, b0, b1);
+        if (s == 0) mman_f16_f32_zero(d, a, b0, b1);
+        else mman_f16_f32(d, a, b0, b1);
     }
 }
 

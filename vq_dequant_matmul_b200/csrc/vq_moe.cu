@@ -200,12 +200,16 @@ constexpr int MOE_MMA_MAX_THREADS = 32 * 9;   // producer warp + 8 consumer warp
 struct MoeMmaArgs {
     Mat W[3];
     int nproj;
-    float *out[3];               // [P][W[p].rows], rows in bucket order
+    int fused;                   // 1: items are (expert, block) of gate W[0] and up W[1]; h = silu(g) * u
+    float *out[3];               // [P][W[p].rows], rows in bucket order (fused: unused)
+    __half *h16;                 // fused: [P][W[0].rows] fp16
     const __half *ain[3];        // A rows: x by token (stage 1) or h by bucket position
     int a_by_token[3];
     const int *sorted, *offsets, *act, *nact;
     int topk;
-    int NW, STAGES, stage_bytes, soff;
+    int NW, STAGES, stage_bytes;
+    int rblk[3];                 // 8-row blocks per item (an item moves a few KB)
+    int soff[3], coff[3];        // offsets in a stage: projection p's codes (coff) and scales (soff)
     int tbl_off[3];              // shared-memory offset of each projection's codebook table
     int tbl_bytes;
     unsigned int *err;
@@ -215,10 +219,18 @@ struct MoeItem {
     int p, e, blk;
 };
 
+__device__ __forceinline__ int moe_blocks(const Mat &W, int rblk) { return (W.rows + MMAV_ROWS * rblk - 1) / (MMAV_ROWS * rblk); }
+
 __device__ __forceinline__ MoeItem moe_item(const MoeMmaArgs &a, int i, int nact) {
     MoeItem it{0, 0, 0};
+    if (a.fused) {
+        const int nb = moe_blocks(a.W[0], a.rblk[0]);
+        it.e = a.act[i / nb];
+        it.blk = i % nb;
+        return it;
+    }
     for (int p = 0; p < a.nproj; p++) {
-        const int nb = (a.W[p].rows + MMAV_ROWS - 1) / MMAV_ROWS;
+        const int nb = moe_blocks(a.W[p], a.rblk[p]);
         if (i < nact * nb) {
             it.p = p;
             it.e = a.act[i / nb];
@@ -230,13 +242,13 @@ __device__ __forceinline__ MoeItem moe_item(const MoeMmaArgs &a, int i, int nact
     return it;
 }
 
-// One item (an 8-row block of one expert's projection) by one warp: every scale group,
-// every token of the expert (16 per pass: the MMA's A rows g and g + 8), and the
-// outputs of its 8 rows.  `stage` holds the block's rows (code_row_bytes apart) and, at
-// `sc`, their scales.
+// One 8-row block of one projection for one chunk of up to 16 of the expert's tokens (the
+// MMA's A rows g and g + 8): tot[0 / 1][0 / 1] = rows 2t / 2t + 1 for token g / g + 8.
+// `stage` holds the block's rows (code_row_bytes apart) and, at `sc`, their scales (both
+// laundered after the stage's wait); x0p / x1p point at the lane's activations.
 template <int D, int BITS>
-__device__ __forceinline__ void moe_warp_item(const MoeMmaArgs &a, const Mat &W, int p, uint32_t stage, uint32_t sc,
-                                              uint32_t cb_lane, int lane, int j0, int j1, int r0)
+__device__ __forceinline__ void moe_block_chunk(const Mat &W, uint32_t stage, uint32_t sc, uint32_t cb_lane, int lane,
+                                                const __half *x0p, const __half *x1p, float (&tot)[2][2])
 {
     constexpr int GB = (64 / D) * BITS / 8;
     const int g = lane >> 2, t = lane & 3;
@@ -244,53 +256,54 @@ __device__ __forceinline__ void moe_warp_item(const MoeMmaArgs &a, const Mat &W,
     const uint32_t crb = (uint32_t)W.code_row_bytes, srow = (uint32_t)W.scale_row_elems * 2;
     const uint32_t row_lane = stage + (uint32_t)g * crb;
     const uint32_t sc0 = sc + (uint32_t)(2 * t) * srow, sc1 = sc0 + srow;   // scales of rows 2t, 2t + 1
-    for (int c0 = j0; c0 < j1; c0 += 16) {
-        const int pos0 = min(c0 + g, j1 - 1), pos1 = min(c0 + g + 8, j1 - 1);
-        const __half *x0p, *x1p;
-        if (a.a_by_token[p]) {
-            x0p = a.ain[p] + (int64_t)(a.sorted[pos0] / a.topk) * W.cols;
-            x1p = a.ain[p] + (int64_t)(a.sorted[pos1] / a.topk) * W.cols;
-        } else {
-            x0p = a.ain[p] + (int64_t)pos0 * W.cols;
-            x1p = a.ain[p] + (int64_t)pos1 * W.cols;
-        }
-        x0p += 16 * t;
-        x1p += 16 * t;
-        float tot[2][2] = {{0.f, 0.f}, {0.f, 0.f}};   // [token g / g + 8][row 2t / 2t + 1]
-        for (int grp = 0; grp < G; grp++) {
-            uint32_t xa[8], xb[8];
-            ldg_x16(x0p + grp * 64, xa);
-            ldg_x16(x1p + grp * 64, xb);
-            float d[4];
-            mma_group<D, BITS>(row_lane + (uint32_t)(grp * GB), t, cb_lane, xa, xb, d);
-            const float s0 = __half2float(__ushort_as_half((unsigned short)lds16(sc0 + 2u * grp)));
-            const float s1 = __half2float(__ushort_as_half((unsigned short)lds16(sc1 + 2u * grp)));
-            tot[0][0] = fmaf(s0, d[0], tot[0][0]);
-            tot[0][1] = fmaf(s1, d[1], tot[0][1]);
-            tot[1][0] = fmaf(s0, d[2], tot[1][0]);
-            tot[1][1] = fmaf(s1, d[3], tot[1][1]);
-        }
-        float *out = a.out[p];
-        const int ra = r0 + 2 * t, rb = ra + 1;
-        if (c0 + g < j1) {
-            if (ra < W.rows) out[(int64_t)(c0 + g) * W.rows + ra] = tot[0][0];
-            if (rb < W.rows) out[(int64_t)(c0 + g) * W.rows + rb] = tot[0][1];
-        }
-        if (c0 + g + 8 < j1) {
-            if (ra < W.rows) out[(int64_t)(c0 + g + 8) * W.rows + ra] = tot[1][0];
-            if (rb < W.rows) out[(int64_t)(c0 + g + 8) * W.rows + rb] = tot[1][1];
-        }
+    tot[0][0] = tot[0][1] = tot[1][0] = tot[1][1] = 0.f;
+#pragma unroll 2
+    for (int grp = 0; grp < G; grp++) {
+        uint32_t xa[8], xb[8];
+        ldg_x16(x0p + grp * 64, xa);
+        ldg_x16(x1p + grp * 64, xb);
+        float d[4];
+        mma_group<D, BITS>(row_lane + (uint32_t)(grp * GB), t, cb_lane, xa, xb, d);
+        const float s0 = __half2float(__ushort_as_half((unsigned short)ldsn16(sc0 + 2u * grp)));
+        const float s1 = __half2float(__ushort_as_half((unsigned short)ldsn16(sc1 + 2u * grp)));
+        tot[0][0] = fmaf(s0, d[0], tot[0][0]);
+        tot[0][1] = fmaf(s1, d[1], tot[0][1]);
+        tot[1][0] = fmaf(s0, d[2], tot[1][0]);
+        tot[1][1] = fmaf(s1, d[3], tot[1][1]);
     }
 }
 
-// Grouped tensor-core GEMV over (projection, active expert, 8-row block) items.  Each CTA
-// takes a balanced contiguous range of items.  Warp 0 (one thread) streams each item's
-// rows and scales into a ring of stages with two bulk copies (an expert's rows are
-// contiguous) and writes the expert's bucket range [j0, j1) into the stage's header;
-// consumer warp w takes items w, w + NW, ..., so the CTA works on NW items at once and no
-// warp waits for another.  Every projection's codebook table stays resident (projections
-// of one launch may be in flight together), so experts must share their tensor's
-// codebook on this path.
+// Dispatch on the projection's geometry (the table's lane copy depends on it).
+__device__ __forceinline__ void moe_block_chunk_any(const Mat &W, uint32_t stage, uint32_t sc, uint32_t tbl, int lane,
+                                                    const __half *x0p, const __half *x1p, float (&tot)[2][2])
+{
+    switch (geom_of(W.d, W.bits)) {
+#define VQ_MOE_CASE(GG, DD, BB)                                                                                 \
+    case GG:                                                                                                  \
+        moe_block_chunk<DD, BB>(W, stage, sc, tbl + (uint32_t)((lane % SmemCB<DD, BB>::NREP) * SmemCB<DD, BB>::ENTRY), \
+                                lane, x0p, x1p, tot);                                                         \
+        break;
+    VQ_MOE_CASE(G_D2_B8, 2, 8)
+    VQ_MOE_CASE(G_D4_B8, 4, 8)
+    VQ_MOE_CASE(G_D8_B8, 8, 8)
+    VQ_MOE_CASE(G_D2_B12, 2, 12)
+    VQ_MOE_CASE(G_D4_B12, 4, 12)
+    VQ_MOE_CASE(G_D8_B12, 8, 12)
+#undef VQ_MOE_CASE
+    default: tot[0][0] = tot[0][1] = tot[1][0] = tot[1][1] = 0.f; break;
+    }
+}
+
+// Grouped tensor-core GEMV over items: (projection, active expert, 8-row block), or in
+// the fused gate/up form (active expert, 8-row block) of both projections, whose warp
+// writes h = fp16(silu(g) * u) directly.  Each CTA takes a balanced contiguous range of
+// items.  Warp 0 (one thread) streams each item's rows and scales into a ring of stages
+// with one bulk copy for the codes and one for the scales of each projection (an
+// expert's rows are contiguous) and writes the expert's bucket range [j0, j1) into the
+// stage's header; consumer warp w takes items w, w + NW, ..., so the CTA works on NW
+// items at once and no warp waits for another.  Every projection's codebook table stays
+// resident (several projections may be in flight together), so experts must share
+// their tensor's codebook on this path.
 __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -303,7 +316,9 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nact = *a.nact;
     int N = 0;
-    for (int p = 0; p < a.nproj; p++) N += nact * ((a.W[p].rows + MMAV_ROWS - 1) / MMAV_ROWS);
+    if (a.fused) N = nact * moe_blocks(a.W[0], a.rblk[0]);
+    else
+        for (int p = 0; p < a.nproj; p++) N += nact * moe_blocks(a.W[p], a.rblk[p]);
     const int i_begin = (int)(((int64_t)N * blockIdx.x) / gridDim.x);
     const int i_end = (int)(((int64_t)N * (blockIdx.x + 1)) / gridDim.x);
     if (i_begin >= i_end) return;                               // uniform over the CTA
@@ -326,18 +341,24 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
                     break;
                 }
                 const MoeItem it = moe_item(a, i, nact);
-                const Mat &W = a.W[it.p];
-                const int r0 = it.blk * MMAV_ROWS;
-                const int nrows = min(MMAV_ROWS, W.rows - r0);
-                const uint8_t *codes = W.codes + (int64_t)it.e * W.expert_code_stride + (int64_t)r0 * W.code_row_bytes;
-                const __half *scales = W.scales + (int64_t)it.e * W.expert_scale_stride + (int64_t)r0 * W.scale_row_elems;
+                const int p0 = a.fused ? 0 : it.p, p1 = a.fused ? 1 : it.p;
+                const int r0 = it.blk * MMAV_ROWS * a.rblk[p0];
+                const int nrows = min(MMAV_ROWS * a.rblk[p0], a.W[p0].rows - r0);
                 hdr[slot] = make_int2(a.offsets[it.e], a.offsets[it.e + 1]);   // published by the arrive below
                 const uint32_t base = smem_u32(sStage + (size_t)slot * a.stage_bytes);
-                const uint32_t cbytes = (uint32_t)(nrows * W.code_row_bytes);
-                const uint32_t sbytes = (uint32_t)(nrows * W.scale_row_elems * 2);
-                mbar_arrive_expect_tx(&full[slot], cbytes + sbytes);
-                bulk_copy_g2s(base, codes, cbytes, &full[slot]);
-                bulk_copy_g2s(base + (uint32_t)a.soff, scales, sbytes, &full[slot]);
+                uint32_t bytes = 0;
+                for (int p = p0; p <= p1; p++)
+                    bytes += (uint32_t)(nrows * (a.W[p].code_row_bytes + a.W[p].scale_row_elems * 2));
+                mbar_arrive_expect_tx(&full[slot], bytes);
+                for (int p = p0; p <= p1; p++) {
+                    const Mat &W = a.W[p];
+                    bulk_copy_g2s(base + (uint32_t)a.coff[p],
+                                  W.codes + (int64_t)it.e * W.expert_code_stride + (int64_t)r0 * W.code_row_bytes,
+                                  (uint32_t)(nrows * W.code_row_bytes), &full[slot]);
+                    bulk_copy_g2s(base + (uint32_t)a.soff[p],
+                                  W.scales + (int64_t)it.e * W.expert_scale_stride + (int64_t)r0 * W.scale_row_elems,
+                                  (uint32_t)(nrows * W.scale_row_elems * 2), &full[slot]);
+                }
             }
         }
         return;
@@ -358,8 +379,11 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
         }
     }
     bar_sync_named(1, nthr);
+    // (laundered: table reads must not move above the barrier)
+    const uint32_t smem_base = launder(smem_u32(smem));
 
     const int cw = warp - 1;
+    const int g = lane >> 2, t = lane & 3;
     for (int i = i_begin + cw, k = cw; i < i_end; i += a.NW, k += a.NW) {
         const int slot = k % a.STAGES, round = k / a.STAGES;
         const bool ok = mbar_wait(&full[slot], round & 1);
@@ -368,26 +392,59 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
             break;
         }
         const MoeItem it = moe_item(a, i, nact);
-        const Mat &W = a.W[it.p];
         const int2 jj = hdr[slot];
-        const uint32_t stage = smem_u32(sStage + (size_t)slot * a.stage_bytes);
-        const uint32_t tbl = smem_u32(smem + a.tbl_off[it.p]);
-        const int r0 = it.blk * MMAV_ROWS;
-        switch (geom_of(W.d, W.bits)) {
-#define VQ_MOE_CASE(GG, DD, BB)                                                                                  \
-    case GG:                                                                                                   \
-        moe_warp_item<DD, BB>(a, W, it.p, stage, stage + (uint32_t)a.soff,                                     \
-                              tbl + (uint32_t)((lane % SmemCB<DD, BB>::NREP) * SmemCB<DD, BB>::ENTRY), lane,   \
-                              jj.x, jj.y, r0);                                                                 \
-        break;
-        VQ_MOE_CASE(G_D2_B8, 2, 8)
-        VQ_MOE_CASE(G_D4_B8, 4, 8)
-        VQ_MOE_CASE(G_D8_B8, 8, 8)
-        VQ_MOE_CASE(G_D2_B12, 2, 12)
-        VQ_MOE_CASE(G_D4_B12, 4, 12)
-        VQ_MOE_CASE(G_D8_B12, 8, 12)
-#undef VQ_MOE_CASE
-        default: break;
+        // (laundered: the stage's loads must not move above the wait)
+        const uint32_t stage = launder(smem_u32(sStage + (size_t)slot * a.stage_bytes));
+        const int pi = a.fused ? 0 : it.p;
+        const Mat &W = a.W[pi];
+        const int nblk = a.rblk[pi];
+        for (int c0 = jj.x; c0 < jj.y; c0 += 16) {
+            const int pos0 = min(c0 + g, jj.y - 1), pos1 = min(c0 + g + 8, jj.y - 1);
+            const __half *x0p, *x1p;
+            if (a.a_by_token[pi]) {
+                x0p = a.ain[pi] + (int64_t)(a.sorted[pos0] / a.topk) * W.cols;
+                x1p = a.ain[pi] + (int64_t)(a.sorted[pos1] / a.topk) * W.cols;
+            } else {
+                x0p = a.ain[pi] + (int64_t)pos0 * W.cols;
+                x1p = a.ain[pi] + (int64_t)pos1 * W.cols;
+            }
+            x0p += 16 * t;
+            x1p += 16 * t;
+            for (int bi = 0; bi < nblk; bi++) {
+                const int r0 = (it.blk * nblk + bi) * MMAV_ROWS;
+                if (r0 >= W.rows) break;
+                const int ra = r0 + 2 * t, rb = ra + 1;
+                float tot[2][2];
+                moe_block_chunk_any(W, stage + (uint32_t)(a.coff[pi] + bi * MMAV_ROWS * (int)W.code_row_bytes),
+                                    stage + (uint32_t)(a.soff[pi] + bi * MMAV_ROWS * (int)W.scale_row_elems * 2),
+                                    smem_base + (uint32_t)a.tbl_off[pi], lane, x0p, x1p, tot);
+                if (a.fused) {
+                    const Mat &U = a.W[1];
+                    float tu[2][2];
+                    moe_block_chunk_any(U, stage + (uint32_t)(a.coff[1] + bi * MMAV_ROWS * (int)U.code_row_bytes),
+                                        stage + (uint32_t)(a.soff[1] + bi * MMAV_ROWS * (int)U.scale_row_elems * 2),
+                                        smem_base + (uint32_t)a.tbl_off[1], lane, x0p, x1p, tu);
+                    // h = fp16(silu(g) * u), as the separate SiLU kernel writes it
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int tok = c0 + g + 8 * h;
+                        if (tok >= jj.y) continue;
+                        if (ra < W.rows)
+                            a.h16[(int64_t)tok * W.rows + ra] = __float2half_rn(tot[h][0] / (1.f + expf(-tot[h][0])) * tu[h][0]);
+                        if (rb < W.rows)
+                            a.h16[(int64_t)tok * W.rows + rb] = __float2half_rn(tot[h][1] / (1.f + expf(-tot[h][1])) * tu[h][1]);
+                    }
+                } else {
+                    float *out = a.out[pi];
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int tok = c0 + g + 8 * h;
+                        if (tok >= jj.y) continue;
+                        if (ra < W.rows) out[(int64_t)tok * W.rows + ra] = tot[h][0];
+                        if (rb < W.rows) out[(int64_t)tok * W.rows + rb] = tot[h][1];
+                    }
+                }
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
@@ -474,9 +531,6 @@ static int moe_num_sms() {
     return n > 0 ? n : 148;
 }
 
-// Shared-memory plan and launch of moe_mma_kernel over the projections in m:
-// UNSUPPORTED (nothing launched) when the tables and a ring of at least 2 * NW stages do
-// not fit, or a projection's scale rows are not whole 16-byte units.
 static size_t moe_table_bytes(const Mat &W) {
     switch (geom_of(W.d, W.bits)) {
     case G_D2_B8: return SmemCB<2, 8>::BYTES;
@@ -488,29 +542,60 @@ static size_t moe_table_bytes(const Mat &W) {
     }
 }
 
-static vq_status launch_moe_mma(MoeMmaArgs &m, cudaStream_t s)
+// Shared-memory plan of moe_mma_kernel: false when it does not apply (scale rows not
+// whole 16-byte units, per-expert codebooks) or the tables and a ring of at least 4
+// stages do not fit.
+static bool plan_moe_mma(MoeMmaArgs &m, size_t *smem_out)
 {
-    int64_t crb = 0, srow = 0;
     size_t tb = 0;
     for (int p = 0; p < m.nproj; p++) {
-        crb = std::max(crb, m.W[p].code_row_bytes);
-        srow = std::max(srow, m.W[p].scale_row_elems * 2);
-        if ((m.W[p].scale_row_elems * 2) % 16 || ((uintptr_t)m.W[p].scales % 16)) return VQ_ERR_UNSUPPORTED;
-        if (m.W[p].num_experts > 1 && (m.W[p].expert_scale_stride * 2) % 16) return VQ_ERR_UNSUPPORTED;
-        if (m.W[p].num_experts > 1 && m.W[p].expert_codebook_stride != 0) return VQ_ERR_UNSUPPORTED;
+        if ((m.W[p].scale_row_elems * 2) % 16 || ((uintptr_t)m.W[p].scales % 16)) return false;
+        if (m.W[p].num_experts > 1 && (m.W[p].expert_scale_stride * 2) % 16) return false;
+        if (m.W[p].num_experts > 1 && m.W[p].expert_codebook_stride != 0) return false;
         m.tbl_off[p] = (int)tb;
         tb += (moe_table_bytes(m.W[p]) + 127) / 128 * 128;
     }
     m.tbl_bytes = (int)tb;
     m.NW = 8;
-    m.soff = (int)(MMAV_ROWS * crb);
-    m.stage_bytes = (int)((MMAV_ROWS * crb + MMAV_ROWS * srow + 127) / 128 * 128);
+    // a stage: the block's codes and scales of every projection it holds (fused: both);
+    // otherwise one projection at a time, sized for the largest
+    // blocks per item: about 4 KB of codes per item (all projections of a fused item)
+    int64_t row_bytes = 0;
+    for (int p = 0; p < (m.fused ? m.nproj : 1); p++) row_bytes += m.W[p].code_row_bytes;
+    for (int p = 0; p < m.nproj; p++) {
+        const int64_t rb = m.fused ? row_bytes : m.W[p].code_row_bytes;
+        int r = 1;
+        while (r < 4 && (int64_t)MMAV_ROWS * 2 * r * rb <= 4096) r *= 2;
+        m.rblk[p] = r;
+    }
+    if (m.fused) m.rblk[1] = m.rblk[0];
+    size_t off = 0, mx = 0;
+    for (int p = 0; p < m.nproj; p++) {
+        const size_t cb = (size_t)MMAV_ROWS * m.rblk[p] * m.W[p].code_row_bytes;
+        const size_t sb = ((size_t)MMAV_ROWS * m.rblk[p] * m.W[p].scale_row_elems * 2 + 15) / 16 * 16;
+        if (m.fused) {
+            m.coff[p] = (int)off;
+            m.soff[p] = (int)(off + cb);
+            off += cb + sb;
+        } else {
+            m.coff[p] = 0;
+            m.soff[p] = (int)cb;
+            mx = std::max(mx, cb + sb);
+        }
+    }
+    m.stage_bytes = (int)(((m.fused ? off : mx) + 127) / 128 * 128);
     const size_t fixed = 128 + tb;
     const size_t per_stage = (size_t)m.stage_bytes + sizeof(int2) + 16;
-    m.STAGES = 32;
-    while (m.STAGES > 2 * m.NW && fixed + (size_t)m.STAGES * per_stage > 232448) m.STAGES--;
+    m.STAGES = 32;   // ideally >= 2 NW (two items in flight per warp); any count is correct
+    while (m.STAGES > 4 && fixed + (size_t)m.STAGES * per_stage > 232448) m.STAGES--;
     const size_t smem = fixed + (size_t)m.STAGES * per_stage;
-    if (smem > 232448) return VQ_ERR_UNSUPPORTED;
+    if (smem > 232448) return false;
+    *smem_out = smem;
+    return true;
+}
+
+static vq_status launch_moe_mma(MoeMmaArgs &m, size_t smem, cudaStream_t s)
+{
     if (cudaFuncSetAttribute(moe_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return VQ_ERR_CUDA;
     moe_mma_kernel<<<moe_num_sms(), 32 * (1 + m.NW), smem, s>>>(m);
@@ -529,18 +614,19 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     auto I = [&](size_t off) { return reinterpret_cast<int *>(W8 + off); };
     auto F = [&](size_t off) { return reinterpret_cast<float *>(W8 + off); };
 
-    // tcgen05 GEMM once experts see several tokens on average, when a projection's scale
-    // rows are not whole 16-byte units (the tensor-core GEMV bulk-copies them), or when
-    // experts have codebooks of their own (the GEMV keeps one table per projection); the
-    // grouped tensor-core GEMV otherwise.
+    // Decode route (few tokens per expert): fused gate/up GEMV, then down GEMV.  The
+    // tcgen05 GEMM once experts see several tokens on average, or when the GEMV does not
+    // apply (scale rows not whole 16-byte units, per-expert codebooks, or shared memory).
     const double per_expert = (double)L.P / std::min(E, L.P);
-    auto srows_ok = [](const Mat &M) {
-        return (M.scale_row_elems * 2) % 16 == 0 && (uintptr_t)M.scales % 16 == 0 &&
-               (M.num_experts == 1 || (M.expert_scale_stride * 2) % 16 == 0);
-    };
-    auto shared_cb = [](const Mat &M) { return M.num_experts == 1 || M.expert_codebook_stride == 0; };
-    const bool use_gemm = per_expert >= 4.0 || !srows_ok(gate) || !srows_ok(up) || !srows_ok(down) ||
-                          !shared_cb(gate) || !shared_cb(up) || !shared_cb(down);
+    MoeMmaArgs m{};
+    m.nproj = 2;
+    m.fused = 1;   // gate and up of a block together: the warp writes h = silu(g) * u
+    m.W[0] = gate; m.W[1] = up;
+    MoeMmaArgs md{};
+    md.nproj = 1;
+    md.W[0] = down;
+    size_t smem1 = 0, smem2 = 0;
+    const bool use_gemm = per_expert >= 4.0 || !plan_moe_mma(m, &smem1) || !plan_moe_mma(md, &smem2);
     const int BT = per_expert <= 24 ? 32 : per_expert <= 48 ? 64 : 128;
 
     BucketArgs b;
@@ -600,27 +686,20 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
         ain1 = xg;
         by_token = 0;
     }
-    MoeMmaArgs m{};
     m.sorted = b.sorted; m.offsets = b.offsets; m.act = b.act; m.nact = b.nact; m.topk = topk;
     m.err = device_error_word();
     if (!m.err) return VQ_ERR_CUDA;
-    m.nproj = 2;
-    m.W[0] = gate; m.W[1] = up;
-    m.out[0] = F(L.g); m.out[1] = F(L.u);
+    __half *h16 = reinterpret_cast<__half *>(W8 + L.h16);
+    m.h16 = h16;
     m.ain[0] = m.ain[1] = ain1;
     m.a_by_token[0] = m.a_by_token[1] = by_token;
-    if ((st = launch_moe_mma(m, s)) != VQ_OK) return st;
-    __half *h16 = reinterpret_cast<__half *>(W8 + L.h16);
-    const int64_t nh = (int64_t)L.P * inter / 4;
-    moe_silu_mul_kernel<<<(unsigned)((nh + 255) / 256), 256, 0, s>>>(F(L.g), F(L.u), b.offsets, E, inter, h16);
-    VQ_CHECK_LAUNCH();
-    MoeMmaArgs md = m;
-    md.nproj = 1;
-    md.W[0] = down;
+    if ((st = launch_moe_mma(m, smem1, s)) != VQ_OK) return st;
+    md.sorted = m.sorted; md.offsets = m.offsets; md.act = m.act; md.nact = m.nact; md.topk = topk;
+    md.err = m.err;
     md.out[0] = F(L.o);
     md.ain[0] = h16;
     md.a_by_token[0] = 0;
-    if ((st = launch_moe_mma(md, s)) != VQ_OK) return st;
+    if ((st = launch_moe_mma(md, smem2, s)) != VQ_OK) return st;
     const int64_t n = (int64_t)T * (hidden / 4);
     moe_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(F(L.o), b.pos, w, T, topk, hidden, y, (int)yt);
     VQ_CHECK_LAUNCH();
