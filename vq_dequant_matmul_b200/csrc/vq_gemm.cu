@@ -310,6 +310,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ GemmArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
+    griddep_wait();   // the activations and (grouped) the tile list are the previous kernel's
     const int z = blockIdx.z;
     const Mat &W = a.W[z];
     const int n0 = blockIdx.y * GEMM_BM;
@@ -339,6 +340,7 @@ vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 // bf16 -> fp16 conversion of the activations (8 elements per thread).
 __global__ void bf16_to_f16_kernel(const __nv_bfloat16 *__restrict__ in, __half *__restrict__ out, int64_t n8)
 {
+    griddep_wait();
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= n8) return;
     uint4 u = __ldg(reinterpret_cast<const uint4 *>(in) + i);
@@ -415,8 +417,7 @@ static vq_status launch_gemm_cfg(const CUtensorMap &map, const GemmArgs &a, int 
     int rows = 0;
     for (int z = 0; z < nproj; z++) rows = std::max(rows, a.W[z].rows);
     dim3 grid(gx, (rows + GEMM_BM - 1) / GEMM_BM, nproj);
-    kern<<<grid, GEMM_THREADS, smem, s>>>(map, a);
-    VQ_CHECK_LAUNCH();
+    if (launch_pdl(kern, grid, dim3(GEMM_THREADS), smem, s, map, a) != cudaSuccess) return VQ_ERR_CUDA;
     return VQ_OK;
 }
 
@@ -481,8 +482,9 @@ vq_status launch_gemm(const Mat &W, const void *x, vq_dtype xt, int M, void *y, 
     const void *x16 = x;
     if (xt == VQ_BF16 && !bf16_tiles) {
         const int64_t n8 = (int64_t)M * W.cols / 8;
-        bf16_to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const __nv_bfloat16 *)x, (__half *)ws, n8);
-        VQ_CHECK_LAUNCH();
+        if (launch_pdl(bf16_to_f16_kernel, dim3((unsigned)((n8 + 255) / 256)), dim3(256), 0, s,
+                       (const __nv_bfloat16 *)x, (__half *)ws, n8) != cudaSuccess)
+            return VQ_ERR_CUDA;
         x16 = ws;
     }
     return run_vq_gemm(a, 1, x16, M, bf16_tiles, dense_bt(M), 0, s);

@@ -324,6 +324,7 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
         mbar_fence_init();
     }
     __syncthreads();
+    griddep_wait();   // inputs and outputs are the previous kernel's until here
 
     auto stage_addr = [&](int slot) -> uint32_t {
         return slot < L.n0 ? A_s0 + (uint32_t)(slot * cfg.SB) : A_s1 + (uint32_t)((slot - L.n0) * cfg.SB);
@@ -398,6 +399,7 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
                 ua = ue;
             }
         }
+        if (lane == 0) griddep_launch_dependents();   // every load is issued: the next kernel may be scheduled
     } else {
         // ---------------- consumers
         const int cw = warp - 1, ctid = threadIdx.x - 32, nct = 32 * NWK;
@@ -650,6 +652,14 @@ void gv_cluster_attr(cudaLaunchConfig_t &lc, cudaLaunchAttribute *at, int C) {
     lc.numAttrs = 1;
 }
 
+// Programmatic dependent launch (see griddep_wait): appended as attribute n of at.
+void gv_pdl_attr(cudaLaunchConfig_t &lc, cudaLaunchAttribute *at, int n) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = (unsigned)(n + 1);
+}
+
 // Tensor maps of one matrix, cached: a map holds only the address, shape, strides and
 // box, so an entry stays valid for any matrix with the same key.
 struct GvMapKey {
@@ -816,12 +826,17 @@ vq_status gv_launch5(const Mat &W, const void *x, int batch, void *y, int yt, Gv
         if (!gv_maps(key, maps)) return VQ_ERR_UNSUPPORTED;
     }
     cudaLaunchConfig_t lc{};
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     lc.gridDim = dim3((unsigned)(c.ncl * c.C));
     lc.blockDim = dim3(gv_threads<NT>());
     lc.dynamicSmemBytes = GV_DYN_SMEM;
     lc.stream = s;
-    if (c.C > 1) gv_cluster_attr(lc, at, c.C);
+    int na = 0;
+    if (c.C > 1) {
+        gv_cluster_attr(lc, at, c.C);
+        na = 1;
+    }
+    gv_pdl_attr(lc, at, na);
     if (cudaLaunchKernelEx(&lc, k, W, (const __half *)x, batch, y, yt, c, maps) != cudaSuccess) return VQ_ERR_CUDA;
     VQ_CHECK_LAUNCH();
     return VQ_OK;

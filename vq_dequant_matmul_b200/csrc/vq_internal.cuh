@@ -60,6 +60,14 @@ template <> __device__ __forceinline__ __half from_f32<__half>(float v) { return
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the previous kernel in the stream is still running; griddep_wait()
+// returns once that kernel has completed and its writes are visible, so it must come
+// before the first access to any input or output.  griddep_launch_dependents() lets the
+// next such kernel be scheduled early (it still waits in its own griddep_wait()).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Store one output element converted to the requested type (runtime switch: the
 // output type only matters in epilogues).
 __device__ __forceinline__ void store_out(void *y, int64_t idx, float v, int yt) {
@@ -88,6 +96,25 @@ __device__ __forceinline__ float group_sum(float v, int width) {
 }
 
 }  // namespace vq
+
+// Launch with programmatic stream serialization (the kernel must call griddep_wait()
+// before touching any input or output).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args)
+{
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, k, static_cast<KArgs>(args)...);
+}
 
 // Host-side launch helpers (status mapping).
 #define VQ_CHECK_LAUNCH()                                              \

@@ -115,6 +115,7 @@ __device__ int block_exclusive_scan(int v, int *sh, int *total)
 
 __global__ void __launch_bounds__(BUCKET_THREADS) moe_bucket_kernel(BucketArgs a)
 {
+    griddep_wait();
     __shared__ int cnt[MOE_MAX_EXPERTS], base[MOE_MAX_EXPERTS], scan_sh[32];
     __shared__ unsigned int bad;
     extern __shared__ unsigned short wcnt_flat[];      // [BUCKET_THREADS / 32][E]
@@ -314,6 +315,7 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
     uint64_t *empty = full + a.STAGES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_wait();   // the bucket lists are the previous kernel's
     const int nact = *a.nact;
     int N = 0;
     if (a.fused) N = nact * moe_blocks(a.W[0], a.rblk[0]);
@@ -458,6 +460,7 @@ template <typename XT>
 __global__ void moe_gather_kernel(const XT *__restrict__ x, const int *__restrict__ sorted, const int *__restrict__ offsets,
                                   int E, int topk, int hidden, __half *__restrict__ xg)
 {
+    griddep_wait();
     const int q = hidden / 8;
     const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const int total = offsets[E];
@@ -481,6 +484,7 @@ __global__ void moe_gather_kernel(const XT *__restrict__ x, const int *__restric
 __global__ void moe_silu_mul_kernel(const float *__restrict__ g, const float *__restrict__ u,
                                     const int *__restrict__ offsets, int E, int inter, __half *__restrict__ h)
 {
+    griddep_wait();
     const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const int64_t n4 = (int64_t)offsets[E] * inter / 4;
     if (idx >= n4) return;
@@ -497,6 +501,7 @@ __global__ void moe_silu_mul_kernel(const float *__restrict__ g, const float *__
 __global__ void moe_combine_kernel(const float *__restrict__ o, const int *__restrict__ pos,
                                    const float *__restrict__ w, int T, int topk, int hidden, void *y, int yt)
 {
+    griddep_wait();
     const int q = hidden / 4;
     const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (idx >= (int64_t)T * q) return;
@@ -598,8 +603,8 @@ static vq_status launch_moe_mma(MoeMmaArgs &m, size_t smem, cudaStream_t s)
 {
     if (cudaFuncSetAttribute(moe_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return VQ_ERR_CUDA;
-    moe_mma_kernel<<<moe_num_sms(), 32 * (1 + m.NW), smem, s>>>(m);
-    VQ_CHECK_LAUNCH();
+    if (launch_pdl(moe_mma_kernel, dim3(moe_num_sms()), dim3(32 * (1 + m.NW)), smem, s, m) != cudaSuccess)
+        return VQ_ERR_CUDA;
     return VQ_OK;
 }
 
@@ -639,8 +644,7 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     if (cudaFuncSetAttribute(moe_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsmem) !=
         cudaSuccess)
         return VQ_ERR_CUDA;
-    moe_bucket_kernel<<<1, BUCKET_THREADS, bsmem, s>>>(b);
-    VQ_CHECK_LAUNCH();
+    if (launch_pdl(moe_bucket_kernel, dim3(1), dim3(BUCKET_THREADS), bsmem, s, b) != cudaSuccess) return VQ_ERR_CUDA;
 
     const int max_active = std::min(E, L.P);
     vq_status st;
@@ -649,10 +653,12 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
         __half *h16 = reinterpret_cast<__half *>(W8 + L.h16);
         const int64_t ng = (int64_t)L.P * (hidden / 8);
         if (xt == VQ_F16)
-            moe_gather_kernel<__half><<<(unsigned)((ng + 255) / 256), 256, 0, s>>>((const __half *)x, b.sorted, b.offsets, E, topk, hidden, xg);
+            st = launch_pdl(moe_gather_kernel<__half>, dim3((unsigned)((ng + 255) / 256)), dim3(256), 0, s,
+                            (const __half *)x, (const int *)b.sorted, (const int *)b.offsets, E, topk, hidden, xg) == cudaSuccess ? VQ_OK : VQ_ERR_CUDA;
         else
-            moe_gather_kernel<__nv_bfloat16><<<(unsigned)((ng + 255) / 256), 256, 0, s>>>((const __nv_bfloat16 *)x, b.sorted, b.offsets, E, topk, hidden, xg);
-        VQ_CHECK_LAUNCH();
+            st = launch_pdl(moe_gather_kernel<__nv_bfloat16>, dim3((unsigned)((ng + 255) / 256)), dim3(256), 0, s,
+                            (const __nv_bfloat16 *)x, (const int *)b.sorted, (const int *)b.offsets, E, topk, hidden, xg) == cudaSuccess ? VQ_OK : VQ_ERR_CUDA;
+        if (st != VQ_OK) return st;
         const int max_tiles = std::min(L.max_tiles, (L.P + BT - 1) / BT + E);
         GemmArgs ga{};
         ga.W[0] = gate; ga.W[1] = up;
@@ -662,15 +668,18 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
         ga.t_exp = b.t_exp; ga.t_row = b.t_row; ga.t_cnt = b.t_cnt; ga.ntiles = b.ntiles;
         if ((st = run_vq_gemm(ga, 2, xg, L.P, false, BT, max_tiles, s)) != VQ_OK) return st;
         const int64_t nh = (int64_t)L.P * inter / 4;
-        moe_silu_mul_kernel<<<(unsigned)((nh + 255) / 256), 256, 0, s>>>(F(L.g), F(L.u), b.offsets, E, inter, h16);
-        VQ_CHECK_LAUNCH();
+        if (launch_pdl(moe_silu_mul_kernel, dim3((unsigned)((nh + 255) / 256)), dim3(256), 0, s, (const float *)F(L.g),
+                       (const float *)F(L.u), (const int *)b.offsets, E, inter, h16) != cudaSuccess)
+            return VQ_ERR_CUDA;
         GemmArgs gd = ga;
         gd.W[0] = down;
         gd.y[0] = F(L.o);
         gd.ldy[0] = hidden;
         if ((st = run_vq_gemm(gd, 1, h16, L.P, false, BT, max_tiles, s)) != VQ_OK) return st;
         const int64_t n = (int64_t)T * (hidden / 4);
-        moe_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(F(L.o), b.pos, w, T, topk, hidden, y, (int)yt);
+        if (launch_pdl(moe_combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, (const float *)F(L.o),
+                   (const int *)b.pos, w, T, topk, hidden, y, (int)yt) != cudaSuccess)
+        return VQ_ERR_CUDA;
         VQ_CHECK_LAUNCH();
         return VQ_OK;
     }
@@ -680,9 +689,9 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     int by_token = 1;
     if (xt != VQ_F16) {   // bf16 activations: gather and convert to fp16 in bucket order
         __half *xg = reinterpret_cast<__half *>(W8 + L.xg);
-        moe_gather_kernel<__nv_bfloat16><<<(unsigned)((ng + 255) / 256), 256, 0, s>>>(
-            (const __nv_bfloat16 *)x, b.sorted, b.offsets, E, topk, hidden, xg);
-        VQ_CHECK_LAUNCH();
+        if (launch_pdl(moe_gather_kernel<__nv_bfloat16>, dim3((unsigned)((ng + 255) / 256)), dim3(256), 0, s,
+                       (const __nv_bfloat16 *)x, (const int *)b.sorted, (const int *)b.offsets, E, topk, hidden, xg) != cudaSuccess)
+            return VQ_ERR_CUDA;
         ain1 = xg;
         by_token = 0;
     }
@@ -701,7 +710,9 @@ vq_status launch_moe(const Mat &gate, const Mat &up, const Mat &down, const void
     md.a_by_token[0] = 0;
     if ((st = launch_moe_mma(md, smem2, s)) != VQ_OK) return st;
     const int64_t n = (int64_t)T * (hidden / 4);
-    moe_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(F(L.o), b.pos, w, T, topk, hidden, y, (int)yt);
+    if (launch_pdl(moe_combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, (const float *)F(L.o),
+                   (const int *)b.pos, w, T, topk, hidden, y, (int)yt) != cudaSuccess)
+        return VQ_ERR_CUDA;
     VQ_CHECK_LAUNCH();
     return VQ_OK;
 }
