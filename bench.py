@@ -208,8 +208,8 @@ def run_ours(args, rank, world, local_rank):
     blk_ms = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(K)) / K for i in range(2)]
     dec_ms = max_over_ranks(blk_ms[0], world)
     pre_ms = max_over_ranks(blk_ms[1], world)
-    value = sum(dec_bytes) * world / (dec_ms * 1e-3) / 1e9
-    prefill_tflops = sum(pre_flops) * world / (pre_ms * 1e-3) / 1e12
+    value = job_throughput(sum(dec_bytes), dec_ms, world) / 1e9
+    prefill_tflops = job_throughput(sum(pre_flops), pre_ms, world) / 1e12
 
     # context (not the timed region): each projection timed alone, one launch between events
     iso = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(6)]
@@ -362,14 +362,21 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest value over the ranks (device times: the job takes as long as the slowest)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, max_ms, world):
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return units_per_rank * world / (max_ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- oracle arm
