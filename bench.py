@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 
 import workloads as wl  # noqa: E402
 
+GEMV_TRAFFIC_BYTES = 47_420_000.0
 METRIC = "VQ GEMV effective HBM GB/s (% of peak); prefill TFLOP/s; MoE layer tokens/s"
 PREFILL_TOKENS = 2048
 COPIES = 3
@@ -233,7 +234,7 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"kernel": "gemv_mma_kernel<2,8,1,1,1> (mma.sync, 16-row A-operand blocks, TMA stages, 2-4 CTA clusters)",
                 "bound": "hbm", "achieved": round(gemv_gbs, 1),
                 "peak": pk["hbm"], "unit": "GB/s", "frac": round(gemv_gbs / pk["hbm"], 4),
-                "traffic": args.traffic, "peak_source": pk["source"] + " (burst copy)",
+                "traffic": args.traffic or None, "peak_source": pk["source"] + " (burst copy)",
                 "launch_ms": round(blk_ms[0] / 3, 5),
                 "per_projection_isolated_gbs": [round(dec_bytes[i] / (iso_ms[i] * 1e-3) / 1e9, 1) for i in range(3)],
                 "frac_of_nominal_8tbs": round(gemv_gbs / 8000.0, 4)}
@@ -457,8 +458,11 @@ def main():
     ap.add_argument("--moe-iters", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-moe", action="store_true")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="dram bytes per launch of the decode GEMV from an ncu capture")
+    # dram__bytes_read.sum + dram__bytes_write.sum per launch of the decode GEMV, mean of the
+    # gate / up / down launches of one ncu capture of this kernel version
+    # (profiles/gemv_mma_c2_decode.md); pass 0 to report null
+    ap.add_argument("--traffic", type=float, default=GEMV_TRAFFIC_BYTES,
+                    help="dram bytes per launch of the decode GEMV from an ncu capture (0: null)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
