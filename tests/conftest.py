@@ -33,8 +33,14 @@ def pytest_collection_modifyitems(config, items):
 @pytest.fixture(scope="session")
 def vqlib():
     """The CUDA library, built in-tree first if missing or older than its sources."""
-    from vq_dequant_matmul_b200 import build as b
+    import importlib.util
 
+    # build.py by path: importing the package would load the library being rebuilt
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location(
+        "vq_dequant_matmul_b200_build", os.path.join(root, "vq_dequant_matmul_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
     b.build()
     import vq_dequant_matmul_b200 as v
 

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libvq_b200.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with vq_dequant_matmul_b200.build.build() "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python vq_dequant_matmul_b200/build.py` "
                       "(nvcc, sm_100a); there is no CPU fallback")
 
 _lib = ctypes.CDLL(LIB_PATH)
