@@ -161,7 +161,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
             int issued = 0;
             for (int kb = 0; kb < nkb; kb++) {
                 const int s = kb % STAGES, r = kb / STAGES;
-                if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1)) { flag_error(abort_flag); break; }
+                if (r > 0 && !mbar_wait_sleep(&empty[s], (r - 1) & 1)) { flag_error(abort_flag); break; }
                 if (*abort_flag) break;
                 mbar_arrive_expect_tx(&full_b[s], B_TILE_BYTES);
                 tma_load_2d(sB + s * B_TILE_BYTES, xmap, &full_b[s], kb * GEMM_BK, m0);
@@ -179,7 +179,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
             constexpr uint32_t idesc = idesc_f16(GEMM_BM, BT, BF16T);
             for (int kb = 0; kb < nkb; kb++) {
                 const int s = kb % STAGES, r = kb / STAGES;
-                if (!mbar_wait(&full_a[s], r & 1) || !mbar_wait(&full_b[s], r & 1)) {
+                if (!mbar_wait_sleep(&full_a[s], r & 1) || !mbar_wait_sleep(&full_b[s], r & 1)) {
                     flag_error(abort_flag);
                     break;
                 }
@@ -223,7 +223,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
                 const int kb = kb0 + 2 * u;
                 if (kb >= nkb || stop) break;                       // uniform over the warp
                 const int s = kb % STAGES, r = kb / STAGES;
-                const bool ok = r == 0 || mbar_wait(&empty[s], (r - 1) & 1);
+                const bool ok = r == 0 || mbar_wait_sleep(&empty[s], (r - 1) & 1);
                 if (__any_sync(0xffffffffu, !ok || *abort_flag)) {   // warp-uniform exit
                     if (lane == 0) flag_error(abort_flag);
                     stop = true;
@@ -272,7 +272,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
 
         // ---------------- epilogue: TMEM -> registers -> y
         __syncwarp();
-        const bool waited = mbar_wait(acc_bar, 0);
+        const bool waited = mbar_wait_sleep(acc_bar, 0);
         if (!waited) flag_error(abort_flag);
         tc_fence_after();
         if (__all_sync(0xffffffffu, waited && !*abort_flag)) {   // warp-uniform: tcgen05.ld is .sync.aligned

@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
         if (lane == 0) {
             for (int i = i_begin, k = 0; i < i_end; i++, k++) {
                 const int slot = k % a.STAGES, round = k / a.STAGES;
-                if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1)) {
+                if (round > 0 && !mbar_wait_sleep(&empty[slot], (round - 1) & 1)) {
                     atomicExch(a.err, 1u);
                     break;
                 }
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(MOE_MMA_MAX_THREADS, 1) moe_mma_kernel(MoeMmaA
     const int g = lane >> 2, t = lane & 3;
     for (int i = i_begin + cw, k = cw; i < i_end; i += a.NW, k += a.NW) {
         const int slot = k % a.STAGES, round = k / a.STAGES;
-        const bool ok = mbar_wait(&full[slot], round & 1);
+        const bool ok = mbar_wait_sleep(&full[slot], round & 1);
         if (!__all_sync(0xffffffffu, ok)) {
             if (lane == 0) atomicExch(a.err, 1u);
             break;
