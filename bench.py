@@ -40,7 +40,7 @@ sys.path.insert(0, ROOT)
 
 import workloads as wl  # noqa: E402
 
-GEMV_TRAFFIC_BYTES = 47_420_000.0
+GEMV_TRAFFIC_BYTES = 47_408_000.0
 METRIC = "VQ GEMV effective HBM GB/s (% of peak); prefill TFLOP/s; MoE layer tokens/s"
 PREFILL_TOKENS = 2048
 COPIES = 3

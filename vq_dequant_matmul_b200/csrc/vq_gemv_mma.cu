@@ -63,6 +63,7 @@ template <int NT> __host__ __device__ constexpr int gv_nw() { return NT == 2 ? 8
 template <int NT> __host__ __device__ constexpr int gv_threads() { return 32 * (gv_nw<NT>() + 1); }
 constexpr int GV_MAX_STAGES = 10;
 constexpr int GV_MAX_R = 14;                 // reduction buffers
+static_assert(GV_MAX_STAGES <= 32 && GV_MAX_R <= 32, "barriers are initialised one per lane of a warp");
 constexpr int GV_TBL = 65536;                // table region (64 KB)
 constexpr int GV_BAR_BYTES = 512;            // mbarriers + abort word
 constexpr int GV_DYN_SMEM = 232448;          // the per-block opt-in maximum (227 KB)
@@ -313,14 +314,16 @@ gemv_mma_kernel(Mat W, const __half *__restrict__ x, int batch, void *__restrict
     const uint32_t abort_a = A_bars + (uint32_t)((2 * GV_MAX_STAGES + GV_MAX_R + 1) * 8);
     const int S = L.stages, R = L.R;
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; s++) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NWK);
+    if (warp == 0) {   // one barrier of each kind per lane (S, R <= 32)
+        if (lane < S) {
+            mbar_init(&full[lane], 1);
+            mbar_init(&empty[lane], NWK);
         }
-        for (int r = 0; r < R; r++) mbar_init(&red_bar[r], NWK);
-        mbar_init(setup_bar, 1);
-        *reinterpret_cast<volatile uint32_t *>(sptr(abort_a)) = 0u;
+        if (lane < R) mbar_init(&red_bar[lane], NWK);
+        if (lane == 0) {
+            mbar_init(setup_bar, 1);
+            *reinterpret_cast<volatile uint32_t *>(sptr(abort_a)) = 0u;
+        }
         mbar_fence_init();
     }
     __syncthreads();
