@@ -11,9 +11,14 @@
 //     expanded weight is used by BT tokens;
 //   * warp 0 (one thread) streams activation tiles [BT][64] into shared memory with TMA
 //     (128-byte swizzle);
-//   * warps 2-9 (256 threads, two per weight row, taking alternate 64-column stages, so
-//     each thread's code prefetch runs several stages ahead) read the row's packed codes and
-//     scale straight from global memory, look the codes up in the shared-memory
+//   * where a row's codes for one 64-column stage are a whole number of 16-byte units
+//     (d = 2 and d = 4 with 8-bit codes, d = 2 with 12-bit codes) the same TMA thread
+//     loads the stage's [128 rows][code bytes] block with the activation tile, on the
+//     same barrier; other geometries read the codes from global memory per thread;
+//   * warps 2-13 (384 threads, three per weight row, each taking every third 64-column
+//     stage, so each thread's prefetch runs several stages ahead and three expansions are
+//     in flight per row) read the row's codes (shared
+//     memory or global) and its scale (global), look the codes up in the shared-memory
 //     codebook and multiply by the scale (one rounding to the tile type).  The expanded
 //     128 x 64 tile goes to tensor memory: each thread writes its row (a warp may only
 //     reach its own 32-lane quarter, so row = 32 (warp mod 4) + lane) as 32 columns with
@@ -23,10 +28,12 @@
 //   * warp 1 (one thread) issues tcgen05.mma (kind::f16, A from tensor memory, B from
 //     shared memory, fp32 accumulation in tensor memory) for each 64-column stage and
 //     frees the stage with tcgen05.commit;
-//   * after the last stage, warps 2-9 read the accumulator out of tensor memory
-//     (tcgen05.ld; two warps per 32-lane quarter, each half of the columns) and store y.
+//   * after the last stage, warps 2-13 read the accumulator out of tensor memory
+//     (tcgen05.ld; the three warps of a 32-lane quarter share the columns) and store y.
 // Stages are a ring of STAGES buffers guarded by mbarriers; every wait is bounded and a
 // wait that runs out sets the library's device error word instead of hanging.
+#include <string.h>
+
 #include <algorithm>
 
 #include "vq_codebook.cuh"
@@ -40,7 +47,17 @@ __device__ unsigned int g_device_error;   // nonzero after a bounded wait ran ou
 
 constexpr int GEMM_BM = 128;       // weight rows per tile (UMMA M)
 constexpr int GEMM_BK = 64;        // columns per stage (one 128-byte swizzle row of 16-bit)
-constexpr int GEMM_THREADS = 320;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 expansion + epilogue
+constexpr int GEMM_NPAR = 3;      // expansion warp groups (each expands every GEMM_NPAR-th stage)
+constexpr int GEMM_THREADS = 64 + 128 * GEMM_NPAR;   // warp 0 TMA, warp 1 MMA + TMEM, then the expansion + epilogue warps
+
+// Code blocks go through TMA when a row's codes for one stage are whole 16-byte units.
+__host__ __device__ constexpr bool gemm_code_tma(int d, int bits) { return ((64 / d) * bits / 8) % 16 == 0; }
+
+// Tensor maps of the projections' codes (used where gemm_code_tma holds): uint8
+// [experts][rows][code_row_bytes], box [1][128][code bytes of one stage].
+struct GemmCodeMaps {
+    CUtensorMap code[2];
+};
 
 // Packed codes of one row for one 64-column stage: 64/d codes.
 template <int D, int BITS>
@@ -66,6 +83,15 @@ struct CodeBlock {
         } else {
 #pragma unroll
             for (int v = 0; v < WORDS; v++) w[v] = __ldg(reinterpret_cast<const uint32_t *>(p) + v);
+        }
+    }
+    // From a 16-byte aligned shared-memory copy of the row's block (TMA layout).
+    __device__ __forceinline__ void load_smem(const uint8_t *p) {
+        static_assert(BYTES % 16 == 0, "whole 16-byte units");
+#pragma unroll
+        for (int v = 0; v < BYTES / 16; v++) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(p + 16 * v);
+            w[4 * v] = u.x; w[4 * v + 1] = u.y; w[4 * v + 2] = u.z; w[4 * v + 3] = u.w;
         }
     }
     __device__ __forceinline__ void zero() {
@@ -104,12 +130,15 @@ __device__ __forceinline__ void flag_error(volatile int *abort_flag) {
 // One CTA: output tile rows [n0, n0 + 128) of expert e's matrix W against activation rows
 // [m0, m0 + mcount) of the tensor map; y[(m0 + j) * ldy + n] for j < mcount.
 template <int D, int BITS, int BT, int STAGES, bool BF16T>
-__device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, int e, int m0, int mcount,
-                                         int n0, void *__restrict__ y, int64_t ldy, int yt, uint8_t *smem_raw)
+__device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const CUtensorMap *cmap, const Mat &W, int e,
+                                         int m0, int mcount, int n0, void *__restrict__ y, int64_t ldy, int yt,
+                                         uint8_t *smem_raw)
 {
     using CB = SmemCB<D, BITS>;
     using Blk = CodeBlock<D, BITS>;
     constexpr int B_TILE_BYTES = BT * GEMM_BK * 2;
+    constexpr bool TMAC = gemm_code_tma(D, BITS);             // code blocks by TMA
+    constexpr int C_TILE_BYTES = TMAC ? GEMM_BM * Blk::BYTES : 0;
     // tensor memory: fp32 accumulator (one column per token), then one 32-column A tile
     // per stage; the allocation is a power of two
     constexpr uint32_t TMEM_NEED = BT + 32 * STAGES;
@@ -119,7 +148,8 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem;
-    uint8_t *sCB = sB + STAGES * B_TILE_BYTES;
+    uint8_t *sC = sB + STAGES * B_TILE_BYTES;                  // TMAC: [STAGES][128 rows][code bytes]
+    uint8_t *sCB = sC + STAGES * C_TILE_BYTES;
     uint64_t *full_a = reinterpret_cast<uint64_t *>(sCB + CB::BYTES);
     uint64_t *full_b = full_a + STAGES;
     uint64_t *empty = full_b + STAGES;
@@ -158,13 +188,16 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
         // ---------------- TMA producer: activation tiles
         if (lane == 0) {
             tma_prefetch_map(xmap);
+            if constexpr (TMAC) tma_prefetch_map(cmap);
             int issued = 0;
             for (int kb = 0; kb < nkb; kb++) {
                 const int s = kb % STAGES, r = kb / STAGES;
                 if (r > 0 && !mbar_wait_sleep(&empty[s], (r - 1) & 1)) { flag_error(abort_flag); break; }
                 if (*abort_flag) break;
-                mbar_arrive_expect_tx(&full_b[s], B_TILE_BYTES);
+                mbar_arrive_expect_tx(&full_b[s], B_TILE_BYTES + C_TILE_BYTES);
                 tma_load_2d(sB + s * B_TILE_BYTES, xmap, &full_b[s], kb * GEMM_BK, m0);
+                if constexpr (TMAC)   // rows past the end read as zeros
+                    tma_load_3d(smem_u32(sC + s * C_TILE_BYTES), cmap, &full_b[s], kb * Blk::BYTES, n0, e);
                 issued++;
             }
             // On an abort, wait (bounded) for the loads still in flight before leaving.
@@ -197,7 +230,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
     } else {
         // ---------------- expansion: thread t writes weight row n0 + t of every stage
         const int t = 32 * (warp & 3) + lane;    // tile row = tensor-memory lane
-        const int par = (warp - 2) >> 2;         // this thread expands stages kb = par, par + 2, ...
+        const int par = (warp - 2) >> 2;         // this thread expands stages kb = par, par + NPAR, ...
         const int row = n0 + t;
         const bool rv = row < W.rows;
         const uint8_t *crow = codes_e + (int64_t)(rv ? row : 0) * W.code_row_bytes;
@@ -205,25 +238,32 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
         const uint8_t *cbl = sCB + (lane % CB::NREP) * CB::ENTRY;
         const uint32_t tquarter = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's tensor-memory lanes
 
-        // Code blocks and scales of the stages kb = par + 2u (u < PF) are kept in flight in
-        // a register ring; a slot is refilled (PF stages ahead) right after it is expanded.
+        // Scales (and, without TMAC, code blocks) of the stages kb = par + NPAR u (u < PF) are
+        // kept in flight in a register ring; a slot is refilled (PF stages ahead) right
+        // after it is expanded.  Rows past the end read row 0; their tile rows only reach
+        // accumulator rows that are never stored.
         constexpr int PF = 5;
-        Blk ring[PF];
+        constexpr int PFC = TMAC ? 1 : PF;
+        Blk ring[PFC];
         __half sr[PF];
 #pragma unroll
         for (int u = 0; u < PF; u++) {
-            const int kbu = par + 2 * u;
+            const int kbu = par + GEMM_NPAR * u;
             sr[u] = __float2half(0.f);
-            if (rv && kbu < nkb) { ring[u].load(crow, kbu); sr[u] = srow[kbu]; } else ring[u].zero();
+            if (kbu < nkb) sr[u] = srow[kbu];
+            if constexpr (!TMAC) {
+                if (kbu < nkb) ring[u].load(crow, kbu); else ring[u].zero();
+            }
         }
         bool stop = false;
-        for (int kb0 = par; kb0 < nkb && !stop; kb0 += 2 * PF) {
+        for (int kb0 = par; kb0 < nkb && !stop; kb0 += GEMM_NPAR * PF) {
 #pragma unroll
             for (int u = 0; u < PF; u++) {
-                const int kb = kb0 + 2 * u;
+                const int kb = kb0 + GEMM_NPAR * u;
                 if (kb >= nkb || stop) break;                       // uniform over the warp
                 const int s = kb % STAGES, r = kb / STAGES;
-                const bool ok = r == 0 || mbar_wait_sleep(&empty[s], (r - 1) & 1);
+                bool ok = r == 0 || mbar_wait_sleep(&empty[s], (r - 1) & 1);
+                if constexpr (TMAC) ok = ok && mbar_wait_sleep(&full_b[s], r & 1);   // the stage's codes landed
                 if (__any_sync(0xffffffffu, !ok || *abort_flag)) {   // warp-uniform exit
                     if (lane == 0) flag_error(abort_flag);
                     stop = true;
@@ -232,7 +272,9 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
                 uint32_t av[32];                                     // the row's 64 tile elements
                 const __half2 s2 = __half2half2(sr[u]);
                 const float sf = __half2float(sr[u]);
-                const Blk &cur = ring[u];
+                Blk tc;
+                if constexpr (TMAC) tc.load_smem(sC + s * C_TILE_BYTES + t * Blk::BYTES);
+                const Blk &cur = TMAC ? tc : ring[u % PFC];
 #pragma unroll
                 for (int c = 0; c < 8; c++) {
                     uint32_t o[4];
@@ -256,7 +298,6 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
                         o[2] = scale_pair<BF16T>(e.z, s2, sf);
                         o[3] = scale_pair<BF16T>(e.w, s2, sf);
                     }
-                    if (!rv) o[0] = o[1] = o[2] = o[3] = 0u;
 #pragma unroll
                     for (int j = 0; j < 4; j++) av[4 * c + j] = o[j];   // column 4c + j: elements 8c + 2j, +1
                 }
@@ -265,8 +306,11 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_a[s]);
-                const int nk = kb + 2 * PF;                          // refill this slot
-                if (rv && nk < nkb) { ring[u].load(crow, nk); sr[u] = srow[nk]; }
+                const int nk = kb + GEMM_NPAR * PF;                  // refill this slot
+                if (nk < nkb) {
+                    sr[u] = srow[nk];
+                    if constexpr (!TMAC) ring[u % PFC].load(crow, nk);
+                }
             }
         }
 
@@ -278,10 +322,9 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
         if (__all_sync(0xffffffffu, waited && !*abort_flag)) {   // warp-uniform: tcgen05.ld is .sync.aligned
             const int q = warp & 3;                  // TMEM lanes 32q..32q+31 belong to this warp
             const int erow = n0 + q * 32 + lane;
-            const int chalf = (warp - 2) >> 2;       // two warps per quarter: each takes half the columns
-            constexpr int CW = BT / 2 >= 32 ? BT / 2 : 32;
+            const int cpar = (warp - 2) >> 2;        // GEMM_NPAR warps per quarter share the columns
 #pragma unroll 1
-            for (int c0 = chalf * CW; c0 < BT && c0 < (chalf + 1) * CW; c0 += 32) {
+            for (int c0 = 32 * cpar; c0 < BT; c0 += 32 * GEMM_NPAR) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
                 tmem_ld_wait();
@@ -307,7 +350,8 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const Mat &W, 
 
 template <int BT, int STAGES, bool BF16T>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ GemmArgs a)
+vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ GemmArgs a,
+               const __grid_constant__ GemmCodeMaps cm)
 {
     extern __shared__ uint8_t smem_raw[];
     griddep_wait();   // the activations and (grouped) the tile list are the previous kernel's
@@ -327,12 +371,12 @@ vq_gemm_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         mcount = min(BT, a.M - m0);
     }
     switch (geom_of(W.d, W.bits)) {
-    case G_D2_B8: gemm_cta<2, 8, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
-    case G_D4_B8: gemm_cta<4, 8, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
-    case G_D8_B8: gemm_cta<8, 8, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
-    case G_D2_B12: gemm_cta<2, 12, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
-    case G_D4_B12: gemm_cta<4, 12, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
-    case G_D8_B12: gemm_cta<8, 12, BT, STAGES, BF16T>(&xmap, W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D2_B8: gemm_cta<2, 8, BT, STAGES, BF16T>(&xmap, &cm.code[z], W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D4_B8: gemm_cta<4, 8, BT, STAGES, BF16T>(&xmap, &cm.code[z], W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D8_B8: gemm_cta<8, 8, BT, STAGES, BF16T>(&xmap, &cm.code[z], W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D2_B12: gemm_cta<2, 12, BT, STAGES, BF16T>(&xmap, &cm.code[z], W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D4_B12: gemm_cta<4, 12, BT, STAGES, BF16T>(&xmap, &cm.code[z], W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
+    case G_D8_B12: gemm_cta<8, 12, BT, STAGES, BF16T>(&xmap, &cm.code[z], W, e, m0, mcount, n0, a.y[z], a.ldy[z], a.yt, smem_raw); break;
     default: break;
     }
 }
@@ -391,9 +435,30 @@ static bool make_x_map(CUtensorMap *map, const void *x, bool bf16, int M, int K,
     return r == CUDA_SUCCESS;
 }
 
-// Shared memory of a launch whose largest codebook table takes cb_bytes.
-static size_t gemm_smem_bytes(int BT, int stages, size_t cb_bytes) {
-    return 1024 + (size_t)stages * ((size_t)BT * GEMM_BK * 2) + cb_bytes + (3 * stages + 1) * 8 + 16;
+// Shared memory of a launch whose largest codebook table takes cb_bytes and whose largest
+// TMA code block takes ct_bytes per stage.
+static size_t gemm_smem_bytes(int BT, int stages, size_t cb_bytes, size_t ct_bytes) {
+    return 1024 + (size_t)stages * ((size_t)BT * GEMM_BK * 2 + ct_bytes) + cb_bytes + (3 * stages + 1) * 8 + 16;
+}
+
+static size_t code_tile_bytes(const Mat &W) {
+    return gemm_code_tma(W.d, W.bits) ? (size_t)GEMM_BM * ((64 / W.d) * W.bits / 8) : 0;
+}
+
+// Code tensor map of W (3-D: bytes of a row, rows, experts).
+static bool make_code_map(CUtensorMap *map, const Mat &W) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const int64_t E = W.num_experts > 1 ? W.num_experts : 1;
+    const int64_t estride = E > 1 ? W.expert_code_stride : W.code_row_bytes * W.rows;
+    cuuint64_t dims[3] = {(cuuint64_t)W.code_row_bytes, (cuuint64_t)W.rows, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)W.code_row_bytes, (cuuint64_t)estride};
+    cuuint32_t box[3] = {(cuuint32_t)((64 / W.d) * W.bits / 8), (cuuint32_t)GEMM_BM, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(W.codes), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 static size_t cb_table_bytes(const Mat &W) {
@@ -408,8 +473,8 @@ static size_t cb_table_bytes(const Mat &W) {
 }
 
 template <int BT, int STAGES, bool BF16T>
-static vq_status launch_gemm_cfg(const CUtensorMap &map, const GemmArgs &a, int nproj, int gx, size_t smem,
-                                 cudaStream_t s)
+static vq_status launch_gemm_cfg(const CUtensorMap &map, const GemmArgs &a, const GemmCodeMaps &cm, int nproj,
+                                 int gx, size_t smem, cudaStream_t s)
 {
     auto kern = vq_gemm_kernel<BT, STAGES, BF16T>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -417,21 +482,28 @@ static vq_status launch_gemm_cfg(const CUtensorMap &map, const GemmArgs &a, int 
     int rows = 0;
     for (int z = 0; z < nproj; z++) rows = std::max(rows, a.W[z].rows);
     dim3 grid(gx, (rows + GEMM_BM - 1) / GEMM_BM, nproj);
-    if (launch_pdl(kern, grid, dim3(GEMM_THREADS), smem, s, map, a) != cudaSuccess) return VQ_ERR_CUDA;
+    if (launch_pdl(kern, grid, dim3(GEMM_THREADS), smem, s, map, a, cm) != cudaSuccess) return VQ_ERR_CUDA;
     return VQ_OK;
 }
 
 template <int BT, bool BF16T>
-static vq_status launch_gemm_bt(const CUtensorMap &map, const GemmArgs &a, int nproj, int gx, cudaStream_t s)
+static vq_status launch_gemm_bt(const CUtensorMap &map, const GemmArgs &a, const GemmCodeMaps &cm, int nproj,
+                                int gx, cudaStream_t s)
 {
-    size_t cb = 0;
-    for (int z = 0; z < nproj; z++) cb = std::max(cb, cb_table_bytes(a.W[z]));
-    if (BT + 32 * 6 <= 512 && gemm_smem_bytes(BT, 6, cb) <= 232448)
-        return launch_gemm_cfg<BT, 6, BF16T>(map, a, nproj, gx, gemm_smem_bytes(BT, 6, cb), s);
-    if (gemm_smem_bytes(BT, 4, cb) <= 232448)
-        return launch_gemm_cfg<BT, 4, BF16T>(map, a, nproj, gx, gemm_smem_bytes(BT, 4, cb), s);
-    if (gemm_smem_bytes(BT, 3, cb) <= 232448)
-        return launch_gemm_cfg<BT, 3, BF16T>(map, a, nproj, gx, gemm_smem_bytes(BT, 3, cb), s);
+    size_t cb = 0, ct = 0;
+    for (int z = 0; z < nproj; z++) {
+        cb = std::max(cb, cb_table_bytes(a.W[z]));
+        ct = std::max(ct, code_tile_bytes(a.W[z]));
+    }
+    // the deepest ring that fits (tensor memory: BT accumulator columns + 32 per stage)
+    if (BT + 32 * 6 <= 512 && gemm_smem_bytes(BT, 6, cb, ct) <= 232448)
+        return launch_gemm_cfg<BT, 6, BF16T>(map, a, cm, nproj, gx, gemm_smem_bytes(BT, 6, cb, ct), s);
+    if (BT + 32 * 5 <= 512 && gemm_smem_bytes(BT, 5, cb, ct) <= 232448)
+        return launch_gemm_cfg<BT, 5, BF16T>(map, a, cm, nproj, gx, gemm_smem_bytes(BT, 5, cb, ct), s);
+    if (gemm_smem_bytes(BT, 4, cb, ct) <= 232448)
+        return launch_gemm_cfg<BT, 4, BF16T>(map, a, cm, nproj, gx, gemm_smem_bytes(BT, 4, cb, ct), s);
+    if (gemm_smem_bytes(BT, 3, cb, ct) <= 232448)
+        return launch_gemm_cfg<BT, 3, BF16T>(map, a, cm, nproj, gx, gemm_smem_bytes(BT, 3, cb, ct), s);
     return VQ_ERR_UNSUPPORTED;
 }
 
@@ -444,19 +516,23 @@ vq_status run_vq_gemm(const GemmArgs &a, int nproj, const void *x16, int x_rows,
     if (!make_x_map(&map, x16, bf16, x_rows, a.W[0].cols, BT)) return VQ_ERR_CUDA;
     const int gx = a.t_exp ? max_tiles : (a.M + BT - 1) / BT;
     if (gx < 1) return VQ_OK;
+    GemmCodeMaps cm;
+    memset(&cm, 0, sizeof(cm));
+    for (int z = 0; z < nproj; z++)
+        if (gemm_code_tma(a.W[z].d, a.W[z].bits) && !make_code_map(&cm.code[z], a.W[z])) return VQ_ERR_UNSUPPORTED;
     if (bf16) {
         switch (BT) {
-        case 32: return launch_gemm_bt<32, true>(map, a, nproj, gx, s);
-        case 64: return launch_gemm_bt<64, true>(map, a, nproj, gx, s);
-        case 128: return launch_gemm_bt<128, true>(map, a, nproj, gx, s);
-        default: return launch_gemm_bt<256, true>(map, a, nproj, gx, s);
+        case 32: return launch_gemm_bt<32, true>(map, a, cm, nproj, gx, s);
+        case 64: return launch_gemm_bt<64, true>(map, a, cm, nproj, gx, s);
+        case 128: return launch_gemm_bt<128, true>(map, a, cm, nproj, gx, s);
+        default: return launch_gemm_bt<256, true>(map, a, cm, nproj, gx, s);
         }
     }
     switch (BT) {
-    case 32: return launch_gemm_bt<32, false>(map, a, nproj, gx, s);
-    case 64: return launch_gemm_bt<64, false>(map, a, nproj, gx, s);
-    case 128: return launch_gemm_bt<128, false>(map, a, nproj, gx, s);
-    default: return launch_gemm_bt<256, false>(map, a, nproj, gx, s);
+    case 32: return launch_gemm_bt<32, false>(map, a, cm, nproj, gx, s);
+    case 64: return launch_gemm_bt<64, false>(map, a, cm, nproj, gx, s);
+    case 128: return launch_gemm_bt<128, false>(map, a, cm, nproj, gx, s);
+    default: return launch_gemm_bt<256, false>(map, a, cm, nproj, gx, s);
     }
 }
 
