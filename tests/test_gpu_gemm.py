@@ -48,7 +48,24 @@ def test_gemm_integer_exact(vqlib, d, bits, M):
 
 
 @pytest.mark.parametrize("d,bits", GEOMS)
-@pytest.mark.parametrize("rows,cols,M", [(128, 64, 40), (200, 320, 256), (384, 1024, 513), (130, 2048, 64)])
+def test_gemm_integer_exact_192_token_tiles(vqlib, d, bits):
+    """2048 weight rows x 512 tokens: on 148 SMs 192-token tiles fill the CTA waves better
+    than 256-token ones (48 vs 32 CTAs), so this shape takes the 192-token tiles, with a
+    ragged last tile of 128 tokens; integer data makes the result exact."""
+    rng = np.random.default_rng(d * 31 + bits)
+    rows, cols, M = 2048, 512, 512
+    pool = rng.integers(-6, 7, (min(1 << bits, 200), d))
+    Wi = pool[rng.integers(0, pool.shape[0], (rows, cols // d))].reshape(rows, cols).astype(np.int64)
+    xi = rng.integers(-8, 9, (M, cols)).astype(np.int64)
+    data = encode_dense(Wi.astype(np.float32), d, bits)
+    W = vqlib.VQMatrix.from_data(data)
+    y = run_gemm(vqlib, W, wl.activation_bits(xi.astype(np.float32), wl.F16), wl.F16)
+    assert np.array_equal(to_np(y), (xi @ Wi.T).astype(np.float64))
+
+
+@pytest.mark.parametrize("d,bits", GEOMS)
+@pytest.mark.parametrize("rows,cols,M", [(128, 64, 40), (200, 320, 256), (384, 1024, 513), (130, 2048, 64),
+                                         (2048, 1024, 500)])
 def test_gemm_vs_oracle(vqlib, d, bits, rows, cols, M):
     data = wl.uniform_tensor(rows, cols, d, bits, seed=rows + cols + M + d)
     x = wl.activations(M, cols, seed=M, dtype=wl.F16)

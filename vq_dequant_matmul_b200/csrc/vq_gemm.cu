@@ -35,6 +35,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "vq_codebook.cuh"
 #include "vq_gemm_api.cuh"
@@ -525,6 +526,7 @@ vq_status run_vq_gemm(const GemmArgs &a, int nproj, const void *x16, int x_rows,
         case 32: return launch_gemm_bt<32, true>(map, a, cm, nproj, gx, s);
         case 64: return launch_gemm_bt<64, true>(map, a, cm, nproj, gx, s);
         case 128: return launch_gemm_bt<128, true>(map, a, cm, nproj, gx, s);
+        case 192: return launch_gemm_bt<192, true>(map, a, cm, nproj, gx, s);
         default: return launch_gemm_bt<256, true>(map, a, cm, nproj, gx, s);
         }
     }
@@ -532,11 +534,35 @@ vq_status run_vq_gemm(const GemmArgs &a, int nproj, const void *x16, int x_rows,
     case 32: return launch_gemm_bt<32, false>(map, a, cm, nproj, gx, s);
     case 64: return launch_gemm_bt<64, false>(map, a, cm, nproj, gx, s);
     case 128: return launch_gemm_bt<128, false>(map, a, cm, nproj, gx, s);
+    case 192: return launch_gemm_bt<192, false>(map, a, cm, nproj, gx, s);
     default: return launch_gemm_bt<256, false>(map, a, cm, nproj, gx, s);
     }
 }
 
-static int dense_bt(int M) { return M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+static int gemm_num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] <= 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+// Tokens per tile of a dense GEMM with M tokens and N weight rows.  Large M: 256 tokens
+// (the most reuse of each expanded weight tile) unless 192-token tiles fill the last wave
+// of CTAs (one per SM) clearly better.
+static int dense_bt(int M, int N) {
+    if (M <= 128) return M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    const int nsm = gemm_num_sms(), rt = (N + GEMM_BM - 1) / GEMM_BM;
+    auto fill = [&](int bt) {
+        const double waves = (double)((M + bt - 1) / bt) * rt / nsm;
+        return waves / std::ceil(waves);
+    };
+    return fill(192) > fill(256) + 0.05 ? 192 : 256;
+}
 
 size_t gemm_workspace_bytes(const Mat &W, vq_dtype xt, int M, uint32_t flags)
 {
@@ -563,7 +589,7 @@ vq_status launch_gemm(const Mat &W, const void *x, vq_dtype xt, int M, void *y, 
             return VQ_ERR_CUDA;
         x16 = ws;
     }
-    return run_vq_gemm(a, 1, x16, M, bf16_tiles, dense_bt(M), 0, s);
+    return run_vq_gemm(a, 1, x16, M, bf16_tiles, dense_bt(M, W.rows), 0, s);
 }
 
 // Device address of the error word on the current device (looked up once per device).
