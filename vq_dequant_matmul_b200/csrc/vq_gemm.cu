@@ -40,6 +40,7 @@
 #include "vq_codebook.cuh"
 #include "vq_gemm_api.cuh"
 #include "vq_internal.cuh"
+#include "vq_mma.cuh"
 #include "vq_sm100.cuh"
 
 namespace vq {
@@ -237,6 +238,13 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const CUtensor
         const uint8_t *crow = codes_e + (int64_t)(rv ? row : 0) * W.code_row_bytes;
         const __half *srow = scales_e + (int64_t)(rv ? row : 0) * W.scale_row_elems;
         const uint8_t *cbl = sCB + (lane % CB::NREP) * CB::ENTRY;
+        // 8-bit codes: the 32-bit shared address of this lane's codebook copy (laundered:
+        // the lookups below must not move above the barrier that published the codebook);
+        // entry e's copies start at e * 128, so one byte permute and a shift give the address
+        const uint32_t cb32 = launder(smem_u32(cbl));
+        auto ent = [&](const Blk &b, int q) -> uint32_t {
+            return cb32 + (__byte_perm(b.w[q >> 2], 0u, 0x4440u | (uint32_t)(q & 3)) << 7);
+        };
         const uint32_t tquarter = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's tensor-memory lanes
 
         // Scales (and, without TMAC, code blocks) of the stages kb = par + NPAR u (u < PF) are
@@ -282,18 +290,21 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap *xmap, const CUtensor
                     if constexpr (D == 2) {
 #pragma unroll
                         for (int j = 0; j < 4; j++) {
-                            const uint32_t e = *reinterpret_cast<const uint32_t *>(cbl + cur.code(4 * c + j) * CB::STRIDE);
+                            const uint32_t e = BITS == 8 ? ldsn32(ent(cur, 4 * c + j))
+                                : *reinterpret_cast<const uint32_t *>(cbl + cur.code(4 * c + j) * CB::STRIDE);
                             o[j] = scale_pair<BF16T>(e, s2, sf);
                         }
                     } else if constexpr (D == 4) {
 #pragma unroll
                         for (int j = 0; j < 2; j++) {
-                            const uint2 e = *reinterpret_cast<const uint2 *>(cbl + cur.code(2 * c + j) * CB::STRIDE);
+                            const uint2 e = BITS == 8 ? ldsn64(ent(cur, 2 * c + j))
+                                : *reinterpret_cast<const uint2 *>(cbl + cur.code(2 * c + j) * CB::STRIDE);
                             o[2 * j] = scale_pair<BF16T>(e.x, s2, sf);
                             o[2 * j + 1] = scale_pair<BF16T>(e.y, s2, sf);
                         }
                     } else {
-                        const uint4 e = *reinterpret_cast<const uint4 *>(cbl + cur.code(c) * CB::STRIDE);
+                        const uint4 e = BITS == 8 ? ldsn128(ent(cur, c))
+                            : *reinterpret_cast<const uint4 *>(cbl + cur.code(c) * CB::STRIDE);
                         o[0] = scale_pair<BF16T>(e.x, s2, sf);
                         o[1] = scale_pair<BF16T>(e.y, s2, sf);
                         o[2] = scale_pair<BF16T>(e.z, s2, sf);
