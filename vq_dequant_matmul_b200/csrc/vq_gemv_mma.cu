@@ -228,7 +228,7 @@ __device__ __forceinline__ void gv_group(uint32_t ra, uint32_t rb, int t, uint32
         }
     } else {
         constexpr uint32_t ENTRY = 2 * D;
-        LaneCodes<D, BITS, true> ca, cb;
+        LaneCodes<D, BITS> ca, cb;
         ca.load(ra, t);
         cb.load(rb, t);
         if constexpr (D == 2) {

@@ -84,11 +84,6 @@ __device__ __forceinline__ uint4 ldg_stream_u4(const void *p) {
     return v;
 }
 
-// Bits [s, s+n) (n <= 32) of the 64-bit value hi:lo, s < 32.
-__device__ __forceinline__ uint32_t funnel_bits(uint32_t lo, uint32_t hi, uint32_t s) {
-    return __funnelshift_r(lo, hi, s);
-}
-
 // Sum of v over the `width` lanes of each aligned lane group (width a power of 2).
 __device__ __forceinline__ float group_sum(float v, int width) {
     for (int off = width >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);

@@ -17,36 +17,7 @@ namespace vq {
 
 constexpr int MMAV_ROWS = 8;   // weight rows per block (the MMA's n)
 
-__device__ __forceinline__ void mma_f16_f32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint32_t lds16(uint32_t a) {
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
-    return v;
-}
-
-// Non-volatile forms for hot loops: the compiler may schedule them freely (overlapping
+// Shared-memory loads in non-volatile form: the compiler may schedule them freely (overlapping
 // the latency of independent loads and MMAs), so their ordering against barriers must
 // come from data dependencies — addresses pass through launder() after the wait that
 // publishes the data, and results pass through consume() before the arrive that frees it.
@@ -100,19 +71,15 @@ __device__ __forceinline__ void bar_sync_named(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-__device__ __forceinline__ void bar_arrive_named(int id, int nthreads) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // The lane's codes of one scale group (64 columns) of its row, as they are needed by
-// the four MMAs: code(j) for j < 64 / d / 4.  NV: non-volatile loads (see ldsn32).
-template <int D, int BITS, bool NV = false>
+// the four MMAs: code(j) for j < 64 / d / 4 (non-volatile loads, see ldsn32).
+template <int D, int BITS>
 struct LaneCodes {
     uint32_t w0, w1, w2;
     int sh;   // 12-bit d = 4 / d = 8: bit offset inside w0:w1
-    static __device__ __forceinline__ uint32_t ld32(uint32_t a) { return NV ? ldsn32(a) : lds32(a); }
-    static __device__ __forceinline__ uint2 ld64(uint32_t a) { return NV ? ldsn64(a) : lds64(a); }
-    static __device__ __forceinline__ uint32_t ld16(uint32_t a) { return NV ? ldsn16(a) : lds16(a); }
+    static __device__ __forceinline__ uint32_t ld32(uint32_t a) { return ldsn32(a); }
+    static __device__ __forceinline__ uint2 ld64(uint32_t a) { return ldsn64(a); }
+    static __device__ __forceinline__ uint32_t ld16(uint32_t a) { return ldsn16(a); }
     __device__ __forceinline__ void load(uint32_t grp_addr, int t) {
         if constexpr (BITS == 8) {
             if constexpr (D == 2) { const uint2 v = ld64(grp_addr + 8 * t); w0 = v.x; w1 = v.y; }
@@ -165,7 +132,7 @@ __device__ __forceinline__ void mma_group(uint32_t codes, int t, uint32_t cb_lan
     // non-volatile loads and MMAs (see ldsn32): `codes` must come from a laundered stage
     // address and `cb_lane` from a laundered table address
     using CB = SmemCB<D, BITS>;
-    LaneCodes<D, BITS, true> lc;
+    LaneCodes<D, BITS> lc;
     lc.load(codes, t);
 #pragma unroll
     for (int s = 0; s < 4; s++) {
@@ -197,12 +164,6 @@ __device__ __forceinline__ void ldg_x16(const __half *p, uint32_t (&x)[8]) {
 __device__ __forceinline__ void ldsn_x16(uint32_t addr, uint32_t (&x)[8]) {
     const uint4 a = ldsn128(addr);
     const uint4 b = ldsn128(addr + 16);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-
-__device__ __forceinline__ void lds_x16(uint32_t addr, uint32_t (&x)[8]) {
-    const uint4 a = lds128(addr);
-    const uint4 b = lds128(addr + 16);
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
