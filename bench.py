@@ -241,7 +241,7 @@ def run_ours(args, rank, world, local_rank):
     gemm_tf = sum(pre_flops) / (blk_ms[1] * 1e-3) / 1e12
     prefill = {"value": round(prefill_tflops, 1), "unit": "TFLOP/s", "ms": round(pre_ms, 4),
                "tokens": M, "flops": sum(pre_flops),
-               "roofline": {"kernel": "vq_gemm_kernel (tcgen05, fp16 tiles)", "bound": "tensor",
+               "roofline": {"kernel": "vq_gemm_kernel<256|192 tokens> (tcgen05, fp16 A tiles in tensor memory, TMA code blocks)", "bound": "tensor",
                             "achieved": round(gemm_tf, 1), "peak": pk["bf16_sus"], "unit": "TFLOP/s",
                             "frac": round(gemm_tf / pk["bf16_sus"], 4),
                             "frac_of_burst_peak": round(gemm_tf / pk["bf16"], 4),
