@@ -80,6 +80,27 @@ def test_gemv_rejects_bad_call(vqlib, args, want):
     assert st == want
 
 
+def test_binding_refuses_host_tensors(vqlib):
+    """The Python binding passes device pointers only: a host tensor is refused before any
+    call into the library (a host address handed to a kernel would fault the GPU)."""
+    import torch
+
+    with pytest.raises(ValueError):
+        vqlib._ptr(torch.zeros(4))
+    assert vqlib._ptr(None) is None
+    cb = torch.zeros((1, 256, 2), dtype=torch.float16)
+    codes = torch.zeros((1, 4, 16), dtype=torch.uint8)
+    sc = torch.zeros((1, 4, 1), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        vqlib.VQMatrix(cb, codes, sc, 4, 64, 2, 8)
+
+    class _W:   # a descriptor stand-in: the activations are checked before the stream is read
+        ptr = None
+
+    with pytest.raises(ValueError):
+        vqlib.vq_gemv(_W(), torch.zeros((1, 64), dtype=torch.float16), torch.zeros((1, 4)))
+
+
 def test_pack_rejects_bad_args(vqlib):
     L = vqlib._lib
     P = ctypes.c_void_p

@@ -85,7 +85,13 @@ def _stream(stream=None):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a CUDA tensor (None passes through as NULL).  Host tensors are
+    refused here: every pointer the library takes is a device pointer."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}: the library takes device pointers only")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def status_string(st: int) -> str:
@@ -125,6 +131,9 @@ class VQMatrix:
                  rows: int, cols: int, d: int, bits: int):
         assert codebook.dtype == torch.float16 and scales.dtype == torch.float16
         assert codes.dtype == torch.uint8 and codes.dim() == 3
+        for t in (codebook, codes, scales):
+            if not t.is_cuda or t.device != codes.device:
+                raise ValueError(f"codebook, codes and scales must be CUDA tensors on one device (got {t.device})")
         self.codebook, self.codes, self.scales = codebook, codes, scales
         self.rows, self.cols, self.d, self.bits = rows, cols, d, bits
         E = codes.shape[0]
