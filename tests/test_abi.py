@@ -80,6 +80,39 @@ def test_gemv_rejects_bad_call(vqlib, args, want):
     assert st == want
 
 
+def test_moe_rejects_bad_args(vqlib):
+    """vq_moe_grouped validates shapes, sizes, alignment and the workspace on the host and
+    launches nothing when they are wrong (fake addresses, never dereferenced)."""
+    L = vqlib._lib
+    P = ctypes.c_void_p
+    E, hidden, inter = 4, 128, 64
+    gate = _mat(vqlib, rows=inter, cols=hidden, num_experts=E, expert_code_stride=inter * 32,
+                expert_scale_stride=inter * 2)
+    up = _mat(vqlib, rows=inter, cols=hidden, num_experts=E, expert_code_stride=inter * 32,
+              expert_scale_stride=inter * 2)
+    down = _mat(vqlib, rows=hidden, cols=inter, scale_row_elems=1, num_experts=E,
+                expert_code_stride=hidden * 32, expert_scale_stride=hidden)
+    n = ctypes.c_size_t(0)
+    assert L.vq_moe_workspace_size(2, 2, E, hidden, inter, ctypes.byref(n)) == 0 and n.value > 0
+
+    def call(g=gate, u=up, dn=down, x=0x40000, xt=0, T=2, ids=0x60000, w=0x70000, topk=2, y=0x80000, yt=2,
+             ws=0x100000, wsb=None):
+        return L.vq_moe_grouped(ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), P(x), xt, T, P(ids), P(w),
+                                topk, P(y), yt, P(ws), n.value if wsb is None else wsb, None)
+
+    assert call(topk=E + 1) == 1                  # more slots than experts
+    assert call(T=0) == 1
+    assert call(x=0) == 1
+    assert call(xt=2) == 1                        # fp32 activations
+    assert call(u=_mat(vqlib, rows=inter + 16, cols=hidden, num_experts=E, expert_code_stride=(inter + 16) * 32,
+                       expert_scale_stride=(inter + 16) * 2)) == 1   # up shape differs from gate
+    assert call(dn=_mat(vqlib, rows=hidden, cols=inter, scale_row_elems=1, num_experts=E - 1,
+                        expert_code_stride=hidden * 32, expert_scale_stride=hidden)) == 1
+    assert call(ws=0x100010) == 3                 # workspace not 256-byte aligned
+    assert call(ids=0x60002) == 3                 # expert ids not 4-byte aligned
+    assert call(wsb=n.value - 1) == 4             # workspace too small
+
+
 def test_binding_refuses_host_tensors(vqlib):
     """The Python binding passes device pointers only: a host tensor is refused before any
     call into the library (a host address handed to a kernel would fault the GPU)."""
