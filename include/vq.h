@@ -116,8 +116,9 @@ vq_status vq_gemv(const vq_matrix *W, const void *x, vq_dtype xt, int32_t batch,
                   void *y, vq_dtype yt, void *ws, size_t ws_bytes, vq_stream_t stream);
 
 /* Prefill GEMM: the same contraction for M >= 1 tokens on the tcgen05 tensor cores.
- * Codes and scales are expanded into fp16 tiles in shared memory and multiplied with
- * fp32 accumulation in tensor memory.  x is [M][cols] (fp16 or bf16, 16-byte aligned,
+ * Codes and scales are expanded into fp16 weight tiles held in tensor memory and
+ * multiplied with fp32 accumulation in tensor memory; the dense weights are never
+ * written to device memory.  x is [M][cols] (fp16 or bf16, 16-byte aligned,
  * cols*2 bytes per row); bf16 activations are first converted to fp16 in the
  * workspace (exact for |x| >= 2^-14).  y is [M][rows] of type yt.
  * Prefill path of the pages: paper §2.5 and §3.4 (prefill-shaped code path). */
